@@ -1,0 +1,227 @@
+"""Python face of the CPU oracle -- TEST INFRASTRUCTURE ONLY.
+
+The storage format (quantise, double-quantise, pack, dequantise) runs in the
+plain C of ``qlora_oracle.c`` through ctypes.  The linear layer is written
+here with numpy in binary64: each product is one ``numpy.matmul`` of the
+bf16 operands upcast exactly to binary64, with no blocking, fusion or
+reordering beyond the definitions.
+
+Forward ("QLoRA", learning-llms.pages.dev/topics/qlora, the forward equation
+h = W^x + (alpha/r) B(Ax) with W^ = dequant(W_4bit)), written for row-major
+activations X [M, K], W [N, K], A [r, K], B [N, r] and s = alpha / r:
+
+    T  = X A^T                       [M, r]
+    Y  = X W^T + s T B^T             [M, N]
+
+Backward ("QLoRA", infra.bea.ai, "The Backward Pass Through Quantization":
+gradients flow through the dequantised frozen base, only the adapters get
+gradients, the NF4 base is never updated):
+
+    G  = dY B                        [M, r]
+    dX = dY W^ + s G A               [M, K]
+    dA = s G^T X                     [r, K]
+    dB = s dY^T T                    [N, r]
+
+T and G stay unrounded (binary64).  There is no bias: the pages show none.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+__all__ = [
+    "BLOCK", "GROUP", "load", "build_oracle", "nf4_levels", "f32_to_bf16",
+    "bf16_to_f32", "absmax_int_quantize", "nf4_nearest", "nf4_sizes",
+    "nf4_quantize", "nf4_dequantize", "linear_fwd", "linear_bwd",
+    "rel_fro", "OracleError",
+]
+
+BLOCK = 64
+GROUP = 256
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "qlora_oracle.c")
+_INC = os.path.join(_HERE, "nf4_levels.inc")
+_LIB = os.path.join(_HERE, "libqlora_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def build_oracle(force: bool = False) -> str:
+    """Compile the plain-C oracle with gcc (no fast-math, no contraction)."""
+    stale = (not os.path.exists(_LIB)
+             or os.path.getmtime(_LIB) < max(os.path.getmtime(_SRC), os.path.getmtime(_INC)))
+    if force or stale:
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+               "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build_oracle()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I64 = ctypes.c_int64
+            lib.oracle_nf4_levels.argtypes = [P]
+            lib.oracle_f32_to_bf16.argtypes = [P, I64, P]
+            lib.oracle_bf16_to_f32.argtypes = [P, I64, P]
+            lib.oracle_absmax_int_quantize.argtypes = [P, I64, ctypes.c_int, P, P]
+            lib.oracle_absmax_int_quantize.restype = ctypes.c_float
+            lib.oracle_nf4_nearest.argtypes = [ctypes.c_float]
+            lib.oracle_nf4_nearest.restype = ctypes.c_int
+            lib.oracle_nf4_sizes.argtypes = [I64, I64, ctypes.c_int, P, P, P]
+            lib.oracle_nf4_quantize.argtypes = [P, I64, I64, ctypes.c_int, P, P, P, P]
+            lib.oracle_nf4_dequantize.argtypes = [P, P, P, P, I64, I64, ctypes.c_int, P]
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ------------------------------------------------------------------ scalars
+
+def nf4_levels() -> np.ndarray:
+    out = np.zeros(16, np.float32)
+    load().oracle_nf4_levels(_ptr(out))
+    return out
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    """binary32 -> bf16 bit patterns (uint16), round to nearest even."""
+    x = np.ascontiguousarray(x, np.float32)
+    out = np.empty(x.shape, np.uint16)
+    load().oracle_f32_to_bf16(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def bf16_to_f32(h: np.ndarray) -> np.ndarray:
+    h = np.ascontiguousarray(h, np.uint16)
+    out = np.empty(h.shape, np.float32)
+    load().oracle_bf16_to_f32(_ptr(h), h.size, _ptr(out))
+    return out
+
+
+def absmax_int_quantize(w: np.ndarray, bits: int = 4):
+    """Symmetric absmax grid of the learning-llms page: returns (q, scale, w_hat)."""
+    w = np.ascontiguousarray(w, np.float32).ravel()
+    q = np.empty(w.size, np.int32)
+    w_hat = np.empty(w.size, np.float32)
+    scale = load().oracle_absmax_int_quantize(_ptr(w), w.size, bits, _ptr(q), _ptr(w_hat))
+    return q, np.float32(scale), w_hat
+
+
+def nf4_nearest(x: float) -> int:
+    return int(load().oracle_nf4_nearest(float(x)))
+
+
+def nf4_sizes(rows: int, cols: int, double_quant: bool = True):
+    c, a, g = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    rc = load().oracle_nf4_sizes(rows, cols, int(double_quant), ctypes.byref(c),
+                                 ctypes.byref(a), ctypes.byref(g))
+    if rc != 0:
+        raise OracleError(f"invalid shape {rows}x{cols}")
+    return c.value, a.value, g.value
+
+
+# ------------------------------------------------------------------ format
+
+def nf4_quantize(w: np.ndarray, double_quant: bool = True) -> dict:
+    """Encode a [rows, cols] matrix (binary32 values; pass bf16 inputs as their
+    exact binary32 upcast).  Returns codes [rows, cols/2] uint8, absmax [blocks]
+    fp32, and with double quantisation q8 [blocks] uint8 and s2 [groups] fp32."""
+    w = np.ascontiguousarray(w, np.float32)
+    rows, cols = w.shape
+    blocks = rows * cols // BLOCK
+    groups = (blocks + GROUP - 1) // GROUP
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    absmax = np.zeros(blocks, np.float32)
+    q8 = np.zeros(blocks, np.uint8) if double_quant else None
+    s2 = np.zeros(groups, np.float32) if double_quant else None
+    rc = load().oracle_nf4_quantize(_ptr(w), rows, cols, int(double_quant), _ptr(codes),
+                                    _ptr(absmax), _ptr(q8), _ptr(s2))
+    if rc == 1:
+        raise OracleError("invalid shape")
+    if rc == 2:
+        raise OracleError("non-finite input")
+    out = {"codes": codes, "absmax": absmax, "rows": rows, "cols": cols,
+           "double_quant": bool(double_quant)}
+    if double_quant:
+        out["q8"] = q8
+        out["s2"] = s2
+    return out
+
+
+def nf4_dequantize(q: dict) -> np.ndarray:
+    """Decode to bf16 bit patterns [rows, cols] (uint16)."""
+    rows, cols = q["rows"], q["cols"]
+    out = np.empty((rows, cols), np.uint16)
+    dq = q["double_quant"]
+    rc = load().oracle_nf4_dequantize(
+        _ptr(np.ascontiguousarray(q["codes"])), _ptr(q.get("q8")) if dq else None,
+        _ptr(q.get("s2")) if dq else None, None if dq else _ptr(q["absmax"]),
+        rows, cols, int(dq), _ptr(out))
+    if rc != 0:
+        raise OracleError("invalid shape")
+    return out
+
+
+# ------------------------------------------------------------- linear layer
+
+def _f64(a: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) or floats -> binary64 (exact)."""
+    if a.dtype == np.uint16:
+        return bf16_to_f32(a).astype(np.float64)
+    return np.asarray(a, np.float64)
+
+
+def linear_fwd(X, W_hat, A, B, alpha: float, r: int):
+    """Returns (Y, T) in binary64.  All operands as bf16 bit patterns or floats."""
+    X, W, A, B = _f64(X), _f64(W_hat), _f64(A), _f64(B)
+    s = float(alpha) / float(r)
+    T = X @ A.T
+    Y = X @ W.T + s * (T @ B.T)
+    return Y, T
+
+
+def linear_bwd(dY, X, W_hat, A, B, alpha: float, r: int, T=None):
+    """Returns dict(dX, dA, dB, G) in binary64.  T is recomputed as X A^T when
+    not given."""
+    dY, X, W, A, B = _f64(dY), _f64(X), _f64(W_hat), _f64(A), _f64(B)
+    s = float(alpha) / float(r)
+    if T is None:
+        T = X @ A.T
+    else:
+        T = np.asarray(T, np.float64)
+    G = dY @ B
+    dX = dY @ W + s * (G @ A)
+    dA = s * (G.T @ X)
+    dB = s * (dY.T @ T)
+    return {"dX": dX, "dA": dA, "dB": dB, "G": G, "T": T}
+
+
+def rel_fro(got, ref) -> float:
+    """Relative Frobenius error ||got - ref|| / ||ref|| in binary64."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.linalg.norm(ref)
+    num = np.linalg.norm(got - ref)
+    return float(num / den) if den > 0 else float(num)

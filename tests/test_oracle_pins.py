@@ -1,0 +1,363 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: numbers
+printed on the pages (tests/golden/, each file citing its source), closed
+forms, invariants, an independent library routine, or brute force.
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from bit_nf4_quantized_21_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_golden(name):
+    kv, rows = {}, []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            try:
+                rows.append([float(p) for p in parts])
+            except ValueError:
+                kv[parts[0]] = parts[1:]
+    return kv, rows
+
+
+# ------------------------------------------------- symmetric int4 (page 1)
+
+def test_worked_int4_block_matches_page():
+    kv, rows = _read_golden("int4_worked_block.txt")
+    w = np.array([r[0] for r in rows], np.float32)
+    q, scale, w_hat = O.absmax_int_quantize(w, bits=4)
+    assert round(float(scale), 4) == float(kv["scale"][0])
+    for i, r in enumerate(rows):
+        assert round(float(w[i] / scale), 2) == pytest.approx(r[1], abs=1e-9)
+        assert q[i] == int(r[2])
+        assert round(float(w_hat[i]), 3) == pytest.approx(r[3], abs=1e-9)
+        assert round(float(w[i] - w_hat[i]), 3) == pytest.approx(r[4], abs=1e-9)
+    err = np.abs(w - w_hat)
+    assert round(float(err.mean()), 3) == float(kv["mean_abs_error"][0])
+    assert round(float(scale / 2), 3) == float(kv["half_step"][0])
+    assert err.max() <= scale / 2
+
+
+def test_outlier_block_matches_page():
+    kv, _ = _read_golden("int4_outlier_block.txt")
+    w = np.array([float(v) for v in kv["w"]], np.float32)
+    _, scale0, _ = O.absmax_int_quantize(np.array(
+        [0.42, -0.31, 0.07, -0.18, 0.55, -0.44, 0.12, -0.09], np.float32), bits=4)
+    q, scale, w_hat = O.absmax_int_quantize(w, bits=4)
+    assert round(float(scale), 3) == float(kv["scale"][0])
+    assert round(float(np.abs(w - w_hat).mean()), 3) == float(kv["mean_abs_error"][0])
+    assert round(float(scale / scale0), 1) == float(kv["coarser_ratio"][0])
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_int_grid_error_at_most_half_step(bits):
+    # "the gap w - w^ is quantization error, at worst half a grid step"
+    for seed in range(10):
+        w = inputs.normal((64,), 1.0, seed, dtype=torch.float32).numpy()
+        q, scale, w_hat = O.absmax_int_quantize(w, bits=bits)
+        assert np.all(np.abs(w - w_hat) <= scale / 2 * (1 + 1e-6))
+        assert q.max() <= 2 ** (bits - 1) - 1 and q.min() >= -(2 ** (bits - 1))
+
+
+def test_int4_widget_statistics_and_spread():
+    kv, _ = _read_golden("int4_widget.txt")
+    n = int(float(kv["n_weights"][0]))
+    means, worsts, ratios = [], [], []
+    for seed in range(20):
+        w = inputs.normal((n,), 1.0, seed, dtype=torch.float32).numpy()
+        _, s4, h4 = O.absmax_int_quantize(w, bits=4)
+        _, s8, h8 = O.absmax_int_quantize(w, bits=8)
+        e4, e8 = np.abs(w - h4), np.abs(w - h8)
+        assert e4.max() <= s4 / 2 * (1 + 1e-6)
+        means.append(e4.mean())
+        worsts.append(e4.max())
+        ratios.append(e4.mean() / e8.mean())
+    # statistical consistency with the widget's sample (its values are not printed)
+    assert abs(np.mean(means) - float(kv["mean_abs_error"][0])) < 0.012
+    assert abs(np.mean(worsts) - float(kv["worst_error"][0])) < 0.03
+    # "~18x wider": the step ratio is 127/7 exactly; measured mean-error ratio near it
+    assert round(127 / 7) == int(float(kv["int4_vs_int8_spread"][0]))
+    assert abs(np.mean(ratios) - 127 / 7) < 1.5
+
+
+# ------------------------------------------------------------ NF4 codebook
+
+def test_nf4_codebook_construction_independent_routine():
+    from scipy.special import ndtri  # a second, independent inverse normal CDF
+    delta = 1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0)
+    pos = ndtri(np.linspace(delta, 0.5, 9)[:8])
+    neg = -ndtri(np.linspace(delta, 0.5, 8)[:7])
+    ref = np.sort(np.concatenate([pos, neg, [0.0]]))
+    ref = (ref / np.abs(ref).max()).astype(np.float32)
+    lv = O.nf4_levels()
+    ulp = np.spacing(np.abs(ref).astype(np.float32))
+    assert np.all(np.abs(lv - ref) <= ulp)
+
+
+def test_nf4_codebook_invariants():
+    lv = O.nf4_levels().astype(np.float64)
+    assert len(set(lv.tolist())) == 16                     # all 16 codes used
+    assert np.all(np.diff(lv) > 0)                         # sorted
+    assert lv[0] == -1.0 and lv[15] == 1.0 and lv[7] == 0.0
+    assert (lv > 0).sum() == 8 and (lv < 0).sum() == 7
+    gaps = np.diff(lv)
+    # dense near zero, sparse in the tails: gaps grow away from zero on each side
+    assert np.all(np.diff(gaps[7:]) > 0)                   # positive side
+    assert np.all(np.diff(gaps[:7]) < 0)                   # negative side
+
+
+def test_nf4_nearest_is_optimal_with_lower_tie():
+    lv = O.nf4_levels().astype(np.float64)
+    rng = np.random.default_rng(0)
+    xs = np.concatenate([rng.uniform(-1.05, 1.05, 4000), lv, -lv]).astype(np.float32)
+    for x in xs:
+        c = O.nf4_nearest(float(x))
+        d = np.abs(float(x) - lv)
+        assert d[c] == d.min()
+        assert c == int(np.argmin(d))                      # first minimum = lower code
+    # exact midpoints that binary32 can hold: the tie goes to the lower code
+    for i in range(15):
+        m = (lv[i] + lv[i + 1]) / 2
+        if float(np.float32(m)) == m:
+            assert O.nf4_nearest(float(m)) == i
+        up = float(np.nextafter(np.float32(m), np.float32(2)))
+        dn = float(np.nextafter(np.float32(m), np.float32(-2)))
+        if up > m:
+            assert O.nf4_nearest(up) == i + 1
+        if dn < m:
+            assert O.nf4_nearest(dn) == i
+
+
+def test_nf4_lower_error_than_uniform_grids():
+    kv, _ = _read_golden("int4_widget.txt")
+    lv = O.nf4_levels().astype(np.float64)
+    red = []
+    for seed in range(20):   # one absmax for 2,048 N(0,1) weights, as in the widget
+        w = inputs.normal((2048,), 1.0, 100 + seed, dtype=torch.float32).numpy()
+        am = np.abs(w).max()
+        codes = np.array([O.nf4_nearest(float(np.float32(v / am))) for v in w])
+        e_nf4 = np.abs(w - lv[codes] * am).mean()
+        _, _, h4 = O.absmax_int_quantize(w, bits=4)
+        red.append(1 - e_nf4 / np.abs(w - h4).mean())
+    r = float(np.mean(red))
+    assert abs(r - float(kv["nf4_error_reduction"][0])) < 0.06, r
+    # 64-weight blocks of N(0, 0.02): NF4 beats int4 and a linspace(-1, 1, 16) grid
+    W = inputs.normal((64, 1024), 0.02, 7, dtype=torch.float32).numpy()
+    q = O.nf4_quantize(W, double_quant=False)
+    w_nf4 = O.bf16_to_f32(O.nf4_dequantize(q)).astype(np.float64)
+    blocks = W.reshape(-1, 64).astype(np.float64)
+    am = np.abs(blocks).max(axis=1, keepdims=True)
+    lin = np.linspace(-1, 1, 16)
+    nearest_lin = lin[np.abs(blocks[..., None] / am[..., None] - lin).argmin(-1)] * am
+    int4 = np.clip(np.rint(blocks / (am / 7)), -8, 7) * (am / 7)
+    e_nf4 = np.abs(W.astype(np.float64) - w_nf4).mean()
+    assert e_nf4 < np.abs(blocks - int4).mean()
+    assert e_nf4 < np.abs(blocks - nearest_lin).mean()
+
+
+# ------------------------------------------------------- NF4 storage format
+
+def test_pack_order_hand_example():
+    kv, _ = _read_golden("nf4_pack_example.txt")
+    want = bytes(int(b, 16) for b in kv["bytes"])
+    lv = O.nf4_levels()
+    w = np.tile(lv, 4).reshape(1, 64).astype(np.float32)
+    q = O.nf4_quantize(w, double_quant=True)
+    assert q["codes"].tobytes() == want
+    assert q["absmax"][0] == 1.0 and q["q8"][0] == 255
+    assert q["s2"][0] == np.float32(1.0) / np.float32(255.0)
+
+
+def test_zero_block_and_tiny_block():
+    w = np.zeros((2, 128), np.float32)
+    w[1, 64:] = np.float32(1e-40)            # a subnormal absmax counts as a zero block
+    w[1, :64] = inputs.normal((64,), 0.02, 1, dtype=torch.float32).numpy()
+    q = O.nf4_quantize(w, double_quant=True)
+    assert np.all(q["codes"][0] == 0x77)
+    assert np.all(q["codes"][1, 32:] == 0x77)
+    deq = O.bf16_to_f32(O.nf4_dequantize(q))
+    assert np.all(deq[0] == 0) and np.all(deq[1, 64:] == 0)
+    allzero = O.nf4_quantize(np.zeros((1, 256), np.float32))
+    assert np.all(allzero["q8"] == 0) and allzero["s2"][0] == 0
+
+
+def test_nonfinite_rejected():
+    for bad in (np.inf, -np.inf, np.nan):
+        w = np.zeros((1, 64), np.float32)
+        w[0, 5] = bad
+        with pytest.raises(O.OracleError):
+            O.nf4_quantize(w)
+
+
+def test_double_quant_bounds_and_group_layout():
+    # K = 11008 gives 172 blocks per row, so 256-block groups straddle rows
+    W = inputs.weight((6, 11008), 0.02, 11, dtype=torch.float32, outlier_frac=1e-3).numpy()
+    q = O.nf4_quantize(W, double_quant=True)
+    blocks = W.reshape(-1, 64)
+    am = np.abs(blocks).max(axis=1)
+    assert np.array_equal(q["absmax"], am)
+    groups = (len(am) + 255) // 256
+    assert len(q["s2"]) == groups
+    for g in range(groups):
+        seg = slice(g * 256, min((g + 1) * 256, len(am)))
+        m = am[seg].max()
+        assert q["s2"][g] == np.float32(m) / np.float32(255)
+        assert q["q8"][seg].max() == 255
+        rec = q["q8"][seg].astype(np.float64) * float(q["s2"][g])
+        assert np.all(np.abs(rec - am[seg]) <= float(q["s2"][g]) * (0.5 + 1e-5))
+
+
+def test_dequant_special_values_and_error_bound():
+    W = inputs.weight((32, 512), 0.02, 12, dtype=torch.float32).numpy()
+    lv = O.nf4_levels().astype(np.float64)
+    for dq in (False, True):
+        q = O.nf4_quantize(W, double_quant=dq)
+        deq = O.bf16_to_f32(O.nf4_dequantize(q)).astype(np.float64).reshape(-1, 64)
+        codes = np.stack([q["codes"] & 0xF, q["codes"] >> 4], -1).reshape(-1, 64)
+        assert np.all(deq[codes == 7] == 0)
+        if dq:
+            scale = (q["q8"].astype(np.float32) * q["s2"][np.arange(len(q["q8"])) // 256]
+                     ).astype(np.float64)
+        else:
+            scale = q["absmax"].astype(np.float64)
+        blocks = W.reshape(-1, 64).astype(np.float64)
+        # the element that sets the absmax decodes to +-scale (levels +-1), in bf16
+        idx = np.abs(blocks).argmax(axis=1)
+        top = deq[np.arange(len(idx)), idx]
+        want = np.sign(blocks[np.arange(len(idx)), idx]) * O.bf16_to_f32(
+            O.f32_to_bf16(scale.astype(np.float32))).astype(np.float64)
+        assert np.array_equal(top, want)
+        if not dq:
+            # nearest-level error bound: half the local gap times absmax, plus bf16 rounding
+            gap = np.diff(lv).max()
+            bound = gap / 2 * scale[:, None] * (1 + 1e-6) + np.abs(deq) * 2.0 ** -8
+            assert np.all(np.abs(blocks - deq) <= bound)
+
+
+def test_bf16_rounding_against_torch():
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.standard_normal(20000).astype(np.float32),
+                        np.array([1.0, 1 + 2 ** -8, 1 + 3 * 2 ** -8, -1 - 2 ** -8,
+                                  3.3895314e38, 1e-40, 0.0, -0.0], np.float32)])
+    mine = O.f32_to_bf16(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(mine, ref)
+
+
+def test_storage_sizes_closed_form():
+    kv, _ = _read_golden("storage_overhead.txt")
+    g = lambda k: float(kv[k][0])
+    for N, K in [(256, 512), (4096, 4096), (11008, 4096), (4096, 11008), (28672, 8192)]:
+        c, a, s = O.nf4_sizes(N, K, True)
+        assert c == N * K // 2 and a == N * K // 64
+        assert s == 4 * math.ceil(N * K / 64 / 256)
+        c0, a0, s0 = O.nf4_sizes(N, K, False)
+        assert a0 == 4 * N * K // 64 and s0 == 0
+    N = K = 4096
+    c, a, s = O.nf4_sizes(N, K, True)
+    bits = 8 * (c + a + s) / (N * K)
+    c0, a0, _ = O.nf4_sizes(N, K, False)
+    bits0 = 8 * (c0 + a0) / (N * K)
+    assert round(bits - 4, 3) == g("overhead_dq_bits")
+    assert bits0 - 4 == g("overhead_fp32_bits") and bits0 == g("total_fp32_bits")
+    assert round(bits0 / 8, 2) == g("total_fp32_bytes")
+    assert round(bits, 2) == g("total_dq_bits")
+    assert round(bits / 8, 2) == g("total_dq_bytes")
+    assert round(bits0 - bits, 2) == g("saved_bits")
+    assert round(65e9 * (bits0 - bits) / 8 / 1e9) == g("saved_65b_gb")
+    assert 8 * a / (N * K) == g("overhead_dq_bits_without_group_scale")
+
+
+# --------------------------------------------------- linear layer identities
+
+def _small_problem(seed=0, M=12, N=40, K=128, r=8):
+    wl = inputs.SINGLE
+    W = inputs.weight((N, K), 0.02, seed, dtype=torch.float32).numpy()
+    q = O.nf4_quantize(W)
+    Wh = O.nf4_dequantize(q)
+    X = inputs.normal((M, K), 1.0, seed + 1).view(torch.int16).numpy().view(np.uint16)
+    dY = inputs.normal((M, N), 1.0, seed + 2).view(torch.int16).numpy().view(np.uint16)
+    A = inputs.normal((r, K), 0.01, seed + 3).view(torch.int16).numpy().view(np.uint16)
+    B = inputs.normal((N, r), 0.01, seed + 4).view(torch.int16).numpy().view(np.uint16)
+    return X, Wh, A, B, dY, wl.alpha, r
+
+
+def test_linear_backward_matches_autograd():
+    X, Wh, A, B, dY, alpha, r = _small_problem()
+    f = lambda a: torch.from_numpy(O.bf16_to_f32(a).astype(np.float64))
+    Xt, Wt, At, Bt, dYt = (f(v) for v in (X, Wh, A, B, dY))
+    Xt.requires_grad_(True); At.requires_grad_(True); Bt.requires_grad_(True)
+    s = alpha / r
+    Y = torch.nn.functional.linear(Xt, Wt) + s * torch.nn.functional.linear(
+        torch.nn.functional.linear(Xt, At), Bt)
+    (Y * dYt).sum().backward()
+    Yo, _ = O.linear_fwd(X, Wh, A, B, alpha, r)
+    g = O.linear_bwd(dY, X, Wh, A, B, alpha, r)
+    assert np.allclose(Yo, Y.detach().numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(g["dX"], Xt.grad.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(g["dA"], At.grad.numpy(), rtol=1e-12, atol=1e-14)
+    assert np.allclose(g["dB"], Bt.grad.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_linear_finite_differences():
+    X, Wh, A, B, dY, alpha, r = _small_problem(seed=5, M=6, N=16, K=64, r=4)
+    x, w, a, b, dy = (O.bf16_to_f32(v).astype(np.float64) for v in (X, Wh, A, B, dY))
+    g = O.linear_bwd(dy, x, w, a, b, alpha, r)
+    loss = lambda x_, a_, b_: float((O.linear_fwd(x_, w, a_, b_, alpha, r)[0] * dy).sum())
+    h = 1e-6
+    rng = np.random.default_rng(1)
+    for _ in range(6):
+        i, k = rng.integers(0, a.shape[0]), rng.integers(0, a.shape[1])
+        ap, am = a.copy(), a.copy(); ap[i, k] += h; am[i, k] -= h
+        assert (loss(x, ap, b) - loss(x, am, b)) / (2 * h) == pytest.approx(g["dA"][i, k], rel=1e-6, abs=1e-9)
+        n, j = rng.integers(0, b.shape[0]), rng.integers(0, b.shape[1])
+        bp, bm = b.copy(), b.copy(); bp[n, j] += h; bm[n, j] -= h
+        assert (loss(x, a, bp) - loss(x, a, bm)) / (2 * h) == pytest.approx(g["dB"][n, j], rel=1e-6, abs=1e-9)
+        m, k2 = rng.integers(0, x.shape[0]), rng.integers(0, x.shape[1])
+        xp, xm = x.copy(), x.copy(); xp[m, k2] += h; xm[m, k2] -= h
+        assert (loss(xp, a, b) - loss(xm, a, b)) / (2 * h) == pytest.approx(g["dX"][m, k2], rel=1e-6, abs=1e-9)
+
+
+def test_linear_special_cases():
+    X, Wh, A, B, dY, alpha, r = _small_problem(seed=9)
+    x = O.bf16_to_f32(X).astype(np.float64)
+    w = O.bf16_to_f32(Wh).astype(np.float64)
+    # B = 0: plain frozen-base GEMM (torch's linear as the second routine)
+    Y0, _ = O.linear_fwd(X, Wh, A, np.zeros_like(B), alpha, r)
+    ref = torch.nn.functional.linear(torch.from_numpy(x), torch.from_numpy(w)).numpy()
+    assert np.allclose(Y0, ref, rtol=1e-13, atol=1e-13)
+    # alpha = 0: no adapter contribution
+    Ya, _ = O.linear_fwd(X, Wh, A, B, 0.0, r)
+    assert np.allclose(Ya, ref, rtol=1e-13, atol=1e-13)
+    # all codes 7: the dequantised base is exactly zero and only the adapter remains
+    q = O.nf4_quantize(np.zeros((Wh.shape[0], Wh.shape[1]), np.float32))
+    Wz = O.nf4_dequantize(q)
+    assert np.all(Wz == 0)
+    Yz, T = O.linear_fwd(X, Wz, A, B, alpha, r)
+    b = O.bf16_to_f32(B).astype(np.float64)
+    assert np.allclose(Yz, alpha / r * (T @ b.T), rtol=1e-13, atol=1e-15)
+
+
+def test_linear_backward_is_linear_in_dY():
+    X, Wh, A, B, dY, alpha, r = _small_problem(seed=13)
+    dy1 = O.bf16_to_f32(dY).astype(np.float64)
+    dy2 = np.roll(dy1, 3, axis=1)
+    g1 = O.linear_bwd(dy1, X, Wh, A, B, alpha, r)
+    g2 = O.linear_bwd(dy2, X, Wh, A, B, alpha, r)
+    g3 = O.linear_bwd(2.0 * dy1 - 0.5 * dy2, X, Wh, A, B, alpha, r)
+    for k in ("dX", "dA", "dB"):
+        assert np.allclose(g3[k], 2.0 * g1[k] - 0.5 * g2[k], rtol=1e-12, atol=1e-13)
