@@ -1,0 +1,13 @@
+"""QLoRA frozen-base NF4 linear layer for NVIDIA B200 (sm_100a).
+
+The compute lives in libqlora.so (hand-written CUDA behind a C ABI,
+include/qlora.h); ``bit_nf4_quantized_21_b200.qlora`` is its ctypes binding
+and ``bit_nf4_quantized_21_b200.inputs`` draws the seeded synthetic inputs.
+The library is loaded on first use; calls raise if it has not been built.
+"""
+from .qlora import (  # noqa: F401
+    NF4Weight, QloraError, empty_nf4, lib, qlora_dequantize, qlora_linear_bwd, qlora_linear_fwd,
+    qlora_nf4_codebook, qlora_nf4_sizes, qlora_quantize_nf4, qlora_workspace_bytes, status_string,
+)
+
+__version__ = "0.1.0"

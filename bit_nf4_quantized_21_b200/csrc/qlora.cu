@@ -1,0 +1,474 @@
+// qlora.cu -- libqlora: the C ABI declared in include/qlora.h.
+//
+// Host side of every entry point: argument validation (before anything is
+// enqueued), tensor-map construction for the TMA loads, workspace carving,
+// and the kernel sequence on the caller's stream.  The only process state is
+// the cached driver entry point for tensor-map encoding and a per-device
+// note that the large-shared-memory kernel attributes are set.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "qlora.h"
+#include "ptx.cuh"
+#include "nf4_constants.cuh"
+#include "nf4_decode.cuh"
+#include "codec.cuh"
+#include "gemm_nf4.cuh"
+#include "skinny.cuh"
+
+using namespace qlora;
+
+namespace {
+
+// ------------------------------------------------------------ small helpers
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t rup(int64_t a, int64_t b) { return cdiv(a, b) * b; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D tensor map: `inner` elements per row (contiguous), `outer` rows,
+// `row_bytes` between rows.  Out-of-bounds boxes are zero-filled.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  std::memset(m, 0, sizeof(*m));
+  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool bf16_map(CUtensorMap* m, const void* p, uint64_t cols, uint64_t rows, uint64_t ld_elems,
+              uint32_t box_c, uint32_t box_r) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p, cols, rows, ld_elems * 2, box_c, box_r,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// kernels with > 48 KB of dynamic shared memory need the opt-in once per device
+bool ensure_smem_attrs() {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load() & bit) return true;
+  const int max_smem = 227 * 1024;
+  bool ok = cudaFuncSetAttribute(k_gemm_nf4<kModeFwd>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_gemm_nf4<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_skinny<0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_skinny<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_skinny<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
+  if (ok) done.fetch_or(bit);
+  return ok;
+}
+
+qlora_status check_launch() {
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------- validation
+qlora_status check_weight(const qlora_nf4_weight* w, bool need_arrays) {
+  if (!w) return QLORA_ERR_INVALID_ARG;
+  if (w->rows < 1 || w->cols < 64 || (w->cols % 64) != 0) return QLORA_ERR_INVALID_ARG;
+  if (w->rows > (int64_t(1) << 31) || w->cols > (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
+  if (w->blocksize != 64 || w->group != 256) return QLORA_ERR_UNSUPPORTED;
+  if (w->reserved != 0 || (w->double_quant != 0 && w->double_quant != 1)) return QLORA_ERR_INVALID_ARG;
+  if (!need_arrays) return QLORA_OK;
+  if (!w->codes || !aligned16(w->codes)) return QLORA_ERR_INVALID_ARG;
+  if (w->double_quant) {
+    if (!w->absmax_q8 || !w->group_scale) return QLORA_ERR_INVALID_ARG;
+  } else {
+    if (!w->absmax_f32 || !aligned16(w->absmax_f32)) return QLORA_ERR_INVALID_ARG;
+  }
+  return QLORA_OK;
+}
+
+// ------------------------------------------------------ skinny planning
+struct SkPlan {
+  int64_t P;
+  int64_t Qtot;
+  int Qn;
+  int qchunks;
+  int num_chunks;
+  int splits;
+  int per_split;
+  int stages;
+  size_t partial_bytes;
+};
+
+SkPlan plan_skinny(int64_t P, int64_t J, int64_t Qtot) {
+  SkPlan pl{};
+  pl.P = P;
+  pl.Qtot = Qtot;
+  pl.Qn = static_cast<int>(std::min<int64_t>(Qtot, 256));
+  pl.qchunks = static_cast<int>(cdiv(Qtot, 256));
+  pl.num_chunks = static_cast<int>(cdiv(J, 64));
+  const int64_t ptiles = cdiv(P, kSkBM);
+  const int64_t target = 2 * 148;
+  int64_t splits = cdiv(target, ptiles * pl.qchunks);
+  splits = std::max<int64_t>(1, std::min<int64_t>(splits, std::max(1, pl.num_chunks / 2)));
+  pl.per_split = static_cast<int>(cdiv(pl.num_chunks, splits));
+  pl.splits = static_cast<int>(cdiv(pl.num_chunks, pl.per_split));
+  const uint32_t stage_bytes = kSkABytes + static_cast<uint32_t>(pl.Qn) * 128u;
+  pl.stages = static_cast<int>(std::max<uint32_t>(2, std::min<uint32_t>(6, (200u * 1024u) / stage_bytes)));
+  pl.partial_bytes = static_cast<size_t>(pl.splits) * P * Qtot * 4;
+  return pl;
+}
+
+size_t skinny_smem(const SkPlan& pl) {
+  return static_cast<size_t>(pl.stages) * (kSkABytes + pl.Qn * 128u) + 1024 + 256;
+}
+
+template <int A_MN, int B_MN>
+qlora_status launch_skinny(const SkPlan& pl, const CUtensorMap& ta, const CUtensorMap& tb, float* partial,
+                           int* status, cudaStream_t st) {
+  SkinnyArgs a{};
+  a.P = pl.P;
+  a.Qn = pl.Qn;
+  a.Qtot = pl.Qtot;
+  a.num_chunks = pl.num_chunks;
+  a.chunks_per_split = pl.per_split;
+  a.stages = pl.stages;
+  a.partial = partial;
+  a.status = status;
+  dim3 grid(static_cast<unsigned>(cdiv(pl.P, kSkBM)), pl.splits, pl.qchunks);
+  k_skinny<A_MN, B_MN><<<grid, kSkThreads, skinny_smem(pl), st>>>(ta, tb, a);
+  return check_launch();
+}
+
+// -------------------------------------------------------- workspace layout
+struct Ws {
+  size_t partial, t32, sx, ghl, thl, bpad, total;
+};
+
+struct Dims {
+  int64_t M, N, K;
+  int r, r8, r16, r64, Qh;
+};
+
+Dims dims_of(int64_t M, int64_t N, int64_t K, int r) {
+  Dims d;
+  d.M = M; d.N = N; d.K = K; d.r = r;
+  d.r8 = static_cast<int>(rup(r, 8));
+  d.r16 = static_cast<int>(rup(r, 16));
+  d.r64 = static_cast<int>(rup(r, 64));
+  d.Qh = static_cast<int>(rup(2 * d.r16, 64));
+  return d;
+}
+
+Ws ws_layout(const Dims& d) {
+  size_t part = 0;
+  part = std::max(part, plan_skinny(d.M, d.K, d.r16).partial_bytes);   // T
+  part = std::max(part, plan_skinny(d.M, d.N, d.r64).partial_bytes);   // G
+  part = std::max(part, plan_skinny(d.K, d.M, d.Qh).partial_bytes);    // dA
+  part = std::max(part, plan_skinny(d.N, d.M, d.Qh).partial_bytes);    // dB
+  auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  Ws w{};
+  size_t off = 0;
+  w.partial = off; off += a256(part);
+  w.t32 = off; off += a256(static_cast<size_t>(d.M) * d.r * 4);
+  w.sx = off; off += a256(static_cast<size_t>(d.M) * d.r8 * 2);
+  w.ghl = off; off += a256(static_cast<size_t>(d.M) * d.Qh * 2);
+  w.thl = off; off += a256(static_cast<size_t>(d.M) * d.Qh * 2);
+  w.bpad = off; off += a256(static_cast<size_t>(d.N) * d.r8 * 2);
+  w.total = off;
+  return w;
+}
+
+qlora_status check_linear(int64_t M, const qlora_nf4_weight* Wq, int r, float alpha, const void* workspace,
+                          size_t ws_bytes) {
+  qlora_status st = check_weight(Wq, true);
+  if (st != QLORA_OK) return st;
+  if (M < 1 || M > (int64_t(1) << 31)) return QLORA_ERR_INVALID_ARG;
+  if (r < 1 || r > 256) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  if (Wq->rows % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  if (ws_bytes < ws_layout(dims_of(M, Wq->rows, Wq->cols, r)).total) return QLORA_ERR_WORKSPACE;
+  return QLORA_OK;
+}
+
+// Finish a token-indexed skinny result (T or G).
+qlora_status finish_rows(const float* src, int64_t src_ld, int splits, int64_t split_stride, const Dims& d,
+                         float s, float* f32, __nv_bfloat16* s_bf16, __nv_bfloat16* hl, cudaStream_t st) {
+  const int width = std::max(d.r16, d.Qh - 2 * d.r16);
+  const int64_t n = d.M * width;
+  k_finish_rows<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, st>>>(src, src_ld, splits, split_stride, d.M, d.r,
+                                                                     d.r8, d.r16, d.Qh, s, f32, s_bf16, hl);
+  return check_launch();
+}
+
+// T = X A^T  (fp32 into t32, and optionally s*T in bf16 into sx).
+qlora_status run_T(const void* X, const void* A, const Dims& d, float s, uint8_t* ws, const Ws& L, float* t32,
+                   __nv_bfloat16* sx, int* status, cudaStream_t st) {
+  SkPlan pl = plan_skinny(d.M, d.K, d.r16);
+  CUtensorMap ta, tb;
+  if (!bf16_map(&ta, X, d.K, d.M, d.K, 64, kSkBM)) return QLORA_ERR_CUDA;
+  if (!bf16_map(&tb, A, d.K, d.r, d.K, 64, static_cast<uint32_t>(pl.Qn))) return QLORA_ERR_CUDA;
+  float* partial = reinterpret_cast<float*>(ws + L.partial);
+  qlora_status rc = launch_skinny<0, 0>(pl, ta, tb, partial, status, st);
+  if (rc != QLORA_OK) return rc;
+  return finish_rows(partial, pl.Qtot, pl.splits, pl.P * pl.Qtot, d, s, t32, sx, nullptr, st);
+}
+
+const void* padded_B(const void* B, const Dims& d, uint8_t* ws, const Ws& L, cudaStream_t st, qlora_status* rc) {
+  *rc = QLORA_OK;
+  if (d.r % 8 == 0) return B;
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(ws + L.bpad);
+  const int64_t n = d.N * d.r8;
+  k_pad_cols<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(B), d.N, d.r,
+                                                                  d.r8, dst);
+  *rc = check_launch();
+  return dst;
+}
+
+qlora_status launch_gemm(int mode, const CUtensorMap& tact, const CUtensorMap& tcodes, const CUtensorMap& tla,
+                         const CUtensorMap& tlb, const GemmArgs& a, cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>(cdiv(a.out_cols, kGemmBN)), static_cast<unsigned>(cdiv(a.M, kGemmBM)));
+  if (mode == kModeFwd)
+    k_gemm_nf4<kModeFwd><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tact, tcodes, tla, tlb, a);
+  else
+    k_gemm_nf4<kModeDx><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tact, tcodes, tla, tlb, a);
+  return check_launch();
+}
+
+}  // namespace
+
+// =================================================================== ABI
+extern "C" {
+
+const char* qlora_version(void) { return "0.1.0"; }
+
+const char* qlora_status_string(qlora_status s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_NONFINITE: return "non-finite input";
+    case QLORA_ERR_TIMEOUT: return "device wait timed out";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+void qlora_nf4_codebook(float* out16) {
+  if (!out16) return;
+  for (int i = 0; i < 16; ++i) out16[i] = kNF4Level[i];
+}
+
+qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int double_quant, size_t* codes_bytes,
+                             size_t* absmax_bytes, size_t* group_bytes) {
+  if (!codes_bytes || !absmax_bytes || !group_bytes) return QLORA_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 64 || cols % 64 != 0) return QLORA_ERR_INVALID_ARG;
+  if (double_quant != 0 && double_quant != 1) return QLORA_ERR_INVALID_ARG;
+  const int64_t blocks = rows * cols / 64;
+  *codes_bytes = static_cast<size_t>(rows * cols / 2);
+  *absmax_bytes = static_cast<size_t>(double_quant ? blocks : 4 * blocks);
+  *group_bytes = static_cast<size_t>(double_quant ? 4 * cdiv(blocks, 256) : 0);
+  return QLORA_OK;
+}
+
+size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  if (M < 1 || N < 1 || K < 64 || K % 64 != 0 || r < 1 || r > 256) return 0;
+  return ws_layout(dims_of(M, N, K, r)).total;
+}
+
+qlora_status qlora_quantize_nf4(const void* W, qlora_dtype w_dtype, const qlora_nf4_weight* out, int* d_status,
+                                void* stream) {
+  qlora_status st = check_weight(out, true);
+  if (st != QLORA_OK) return st;
+  if (!W || !aligned16(W)) return QLORA_ERR_INVALID_ARG;
+  if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (out->absmax_f32 && !aligned16(out->absmax_f32)) return QLORA_ERR_INVALID_ARG;
+  const int64_t nblocks = out->rows * out->cols / 64;
+  const unsigned groups = static_cast<unsigned>(cdiv(nblocks, 256));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (w_dtype == QLORA_BF16)
+    k_quantize_nf4<__nv_bfloat16><<<groups, kQuantThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(W), nblocks, out->double_quant, out->codes, out->absmax_q8,
+        out->group_scale, out->absmax_f32, d_status);
+  else
+    k_quantize_nf4<float><<<groups, kQuantThreads, 0, s>>>(static_cast<const float*>(W), nblocks,
+                                                           out->double_quant, out->codes, out->absmax_q8,
+                                                           out->group_scale, out->absmax_f32, d_status);
+  return check_launch();
+}
+
+qlora_status qlora_dequantize(const qlora_nf4_weight* Wq, void* W_out, void* stream) {
+  qlora_status st = check_weight(Wq, true);
+  if (st != QLORA_OK) return st;
+  if (!W_out || !aligned16(W_out)) return QLORA_ERR_INVALID_ARG;
+  const int64_t nblocks = Wq->rows * Wq->cols / 64;
+  k_dequantize_nf4<<<static_cast<unsigned>(cdiv(nblocks, kDeqThreads)), kDeqThreads, 0,
+                     static_cast<cudaStream_t>(stream)>>>(Wq->codes, Wq->absmax_q8, Wq->group_scale, Wq->absmax_f32,
+                                                          Wq->double_quant, nblocks,
+                                                          static_cast<__nv_bfloat16*>(W_out));
+  return check_launch();
+}
+
+qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* Wq, const void* A, const void* B,
+                              int r, float alpha, void* Y, float* T_save, void* workspace, size_t ws_bytes,
+                              int* d_status, void* stream) {
+  qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes);
+  if (st != QLORA_OK) return st;
+  if (!X || !A || !B || !Y || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y))
+    return QLORA_ERR_INVALID_ARG;
+  if (T_save && !aligned16(T_save)) return QLORA_ERR_INVALID_ARG;
+  if (!ensure_smem_attrs()) return QLORA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const Dims d = dims_of(M, Wq->rows, Wq->cols, r);
+  const Ws L = ws_layout(d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const float s = alpha / static_cast<float>(r);
+  float* t32 = T_save ? T_save : reinterpret_cast<float*>(ws + L.t32);
+  __nv_bfloat16* sT = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
+
+  // 1. T = X A^T and s*T (bf16) for the fold
+  st = run_T(X, A, d, s, ws, L, t32, sT, d_status, cs);
+  if (st != QLORA_OK) return st;
+  const void* Bp = padded_B(B, d, ws, L, cs, &st);
+  if (st != QLORA_OK) return st;
+
+  // 2. Y = X W^T + (sT) B^T
+  CUtensorMap tact, tcodes, tla, tlb;
+  if (!bf16_map(&tact, X, d.K, d.M, d.K, 64, kGemmBM)) return QLORA_ERR_CUDA;
+  if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 32, kGemmBN,
+                CU_TENSOR_MAP_SWIZZLE_32B))
+    return QLORA_ERR_CUDA;
+  if (!bf16_map(&tla, sT, d.r8, d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
+  if (!bf16_map(&tlb, Bp, d.r8, d.N, d.r8, 64, kGemmBN)) return QLORA_ERR_CUDA;
+  GemmArgs a{};
+  a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
+  a.wN = d.N; a.wK = d.K; a.M = d.M; a.out_cols = d.N; a.ldo = d.N;
+  a.out = static_cast<__nv_bfloat16*>(Y);
+  a.num_kt = static_cast<int>(d.K / 64);
+  a.lora_r16 = d.r16;
+  a.status = d_status;
+  return launch_gemm(kModeFwd, tact, tcodes, tla, tlb, a, cs);
+}
+
+qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const qlora_nf4_weight* Wq, const void* A,
+                              const void* B, int r, float alpha, const float* T_saved, void* dX, void* dA, void* dB,
+                              qlora_dtype grad_dtype, void* workspace, size_t ws_bytes, int* d_status,
+                              void* stream) {
+  qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes);
+  if (st != QLORA_OK) return st;
+  if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(dA) || !aligned16(dB))
+    return QLORA_ERR_INVALID_ARG;
+  if ((dX && !aligned16(dX)) || (T_saved && !aligned16(T_saved))) return QLORA_ERR_INVALID_ARG;
+  if (grad_dtype != QLORA_F32 && grad_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (!ensure_smem_attrs()) return QLORA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const Dims d = dims_of(M, Wq->rows, Wq->cols, r);
+  const Ws L = ws_layout(d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const float s = alpha / static_cast<float>(r);
+  float* partial = reinterpret_cast<float*>(ws + L.partial);
+  __nv_bfloat16* sG = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
+  __nv_bfloat16* Ghl = reinterpret_cast<__nv_bfloat16*>(ws + L.ghl);
+  __nv_bfloat16* Thl = reinterpret_cast<__nv_bfloat16*>(ws + L.thl);
+
+  const void* Bp = padded_B(B, d, ws, L, cs, &st);
+  if (st != QLORA_OK) return st;
+
+  // 1. G = dY B -> s*G (bf16, for the dX fold) and [G_hi | G_lo] (for dA)
+  {
+    SkPlan pl = plan_skinny(d.M, d.N, d.r64);
+    CUtensorMap ta, tb;
+    if (!bf16_map(&ta, dY, d.N, d.M, d.N, 64, kSkBM)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&tb, Bp, d.r8, d.N, d.r8, 64, 64)) return QLORA_ERR_CUDA;
+    st = launch_skinny<0, 1>(pl, ta, tb, partial, d_status, cs);
+    if (st != QLORA_OK) return st;
+    st = finish_rows(partial, pl.Qtot, pl.splits, pl.P * pl.Qtot, d, s, nullptr, sG, Ghl, cs);
+    if (st != QLORA_OK) return st;
+  }
+  // 2. dX = dY W^ + (sG) A
+  if (dX) {
+    CUtensorMap tact, tcodes, tla, tlb;
+    if (!bf16_map(&tact, dY, d.N, d.M, d.N, 64, kGemmBM)) return QLORA_ERR_CUDA;
+    if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 128, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+      return QLORA_ERR_CUDA;
+    if (!bf16_map(&tla, sG, d.r8, d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&tlb, A, d.K, d.r, d.K, 64, 64)) return QLORA_ERR_CUDA;
+    GemmArgs a{};
+    a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
+    a.wN = d.N; a.wK = d.K; a.M = d.M; a.out_cols = d.K; a.ldo = d.K;
+    a.out = static_cast<__nv_bfloat16*>(dX);
+    a.num_kt = static_cast<int>(cdiv(d.N, 64));
+    a.lora_r16 = d.r16;
+    a.status = d_status;
+    st = launch_gemm(kModeDx, tact, tcodes, tla, tlb, a, cs);
+    if (st != QLORA_OK) return st;
+  }
+  // 3. T (saved or recomputed) -> [T_hi | T_lo]
+  {
+    const float* t = T_saved;
+    if (!t) {
+      float* t32 = reinterpret_cast<float*>(ws + L.t32);
+      st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
+      if (st != QLORA_OK) return st;
+      t = t32;
+    }
+    st = finish_rows(t, d.r, 1, 0, d, s, nullptr, nullptr, Thl, cs);
+    if (st != QLORA_OK) return st;
+  }
+  const int out_bf16 = grad_dtype == QLORA_BF16 ? 1 : 0;
+  // 4. dA = s G^T X   (C[k, q] = sum_m X[m, k] Ghl[m, q])
+  {
+    SkPlan pl = plan_skinny(d.K, d.M, d.Qh);
+    CUtensorMap ta, tb;
+    if (!bf16_map(&ta, X, d.K, d.M, d.K, 64, 64)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&tb, Ghl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
+    st = launch_skinny<1, 1>(pl, ta, tb, partial, d_status, cs);
+    if (st != QLORA_OK) return st;
+    dim3 g(static_cast<unsigned>(cdiv(d.K, 32)), static_cast<unsigned>(cdiv(d.r, 32)));
+    k_finish_grad<<<g, 256, 0, cs>>>(partial, pl.Qtot, pl.splits, d.K, d.r, d.r16, s, 1, out_bf16, dA);
+    st = check_launch();
+    if (st != QLORA_OK) return st;
+  }
+  // 5. dB = s dY^T T  (C[n, q] = sum_m dY[m, n] Thl[m, q])
+  {
+    SkPlan pl = plan_skinny(d.N, d.M, d.Qh);
+    CUtensorMap ta, tb;
+    if (!bf16_map(&ta, dY, d.N, d.M, d.N, 64, 64)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&tb, Thl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
+    st = launch_skinny<1, 1>(pl, ta, tb, partial, d_status, cs);
+    if (st != QLORA_OK) return st;
+    dim3 g(static_cast<unsigned>(cdiv(d.N, 32)), static_cast<unsigned>(cdiv(d.r, 32)));
+    k_finish_grad<<<g, 256, 0, cs>>>(partial, pl.Qtot, pl.splits, d.N, d.r, d.r16, s, 0, out_bf16, dB);
+    st = check_launch();
+  }
+  return st;
+}
+
+}  // extern "C"

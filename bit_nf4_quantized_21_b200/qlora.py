@@ -1,0 +1,237 @@
+"""Python binding of libqlora (ctypes): argument marshalling only.
+
+Every function here has the name of the C entry point it calls
+(include/qlora.h) and does nothing but turn torch tensors into device
+pointers, pick up the current CUDA stream, call the library and raise on a
+non-OK status.  There is no fallback path: if libqlora.so is missing, or a
+tensor is not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqlora.so")
+
+QLORA_OK = 0
+QLORA_F32 = 0
+QLORA_BF16 = 1
+DEV_NONFINITE = 1
+DEV_TIMEOUT = 2
+
+EXPORTED = (
+    "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
+    "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
+    "qlora_version",
+)
+
+
+class QloraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class NF4WeightC(ctypes.Structure):
+    _fields_ = [
+        ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+        ("blocksize", ctypes.c_int32), ("group", ctypes.c_int32),
+        ("double_quant", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("codes", ctypes.c_void_p), ("absmax_q8", ctypes.c_void_p),
+        ("group_scale", ctypes.c_void_p), ("absmax_f32", ctypes.c_void_p),
+    ]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqlora.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"libqlora.so not found at {LIB_PATH}; build it with "
+                    "`python -m bit_nf4_quantized_21_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I64, I32, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+            L.qlora_nf4_sizes.argtypes = [I64, I64, I32, P, P, P]
+            L.qlora_nf4_sizes.restype = I32
+            L.qlora_nf4_codebook.argtypes = [P]
+            L.qlora_nf4_codebook.restype = None
+            L.qlora_quantize_nf4.argtypes = [P, I32, ctypes.POINTER(NF4WeightC), P, P]
+            L.qlora_quantize_nf4.restype = I32
+            L.qlora_dequantize.argtypes = [ctypes.POINTER(NF4WeightC), P, P]
+            L.qlora_dequantize.restype = I32
+            L.qlora_workspace_bytes.argtypes = [I64, I64, I64, I32]
+            L.qlora_workspace_bytes.restype = ctypes.c_size_t
+            L.qlora_linear_fwd.argtypes = [P, I64, ctypes.POINTER(NF4WeightC), P, P, I32, F, P, P, P,
+                                           ctypes.c_size_t, P, P]
+            L.qlora_linear_fwd.restype = I32
+            L.qlora_linear_bwd.argtypes = [P, P, I64, ctypes.POINTER(NF4WeightC), P, P, I32, F, P, P,
+                                           P, P, I32, P, ctypes.c_size_t, P, P]
+            L.qlora_linear_bwd.restype = I32
+            L.qlora_status_string.argtypes = [I32]
+            L.qlora_status_string.restype = ctypes.c_char_p
+            L.qlora_version.argtypes = []
+            L.qlora_version.restype = ctypes.c_char_p
+            _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().qlora_status_string(int(s)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != QLORA_OK:
+        raise QloraError(rc, where)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libqlora takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous (row-major)")
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int | None:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+# ------------------------------------------------------------------ weights
+
+@dataclass
+class NF4Weight:
+    """Device arrays of one NF4 weight [rows, cols] (see qlora_nf4_weight)."""
+    rows: int
+    cols: int
+    double_quant: bool
+    codes: torch.Tensor                 # uint8 [rows, cols/2]
+    absmax_q8: torch.Tensor | None      # uint8 [blocks]
+    group_scale: torch.Tensor | None    # fp32 [groups]
+    absmax_f32: torch.Tensor | None     # fp32 [blocks]
+
+    def c(self) -> NF4WeightC:
+        return NF4WeightC(self.rows, self.cols, 64, 256, int(self.double_quant), 0,
+                          _ptr(self.codes), _ptr(self.absmax_q8), _ptr(self.group_scale),
+                          _ptr(self.absmax_f32))
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.codes, self.absmax_q8, self.group_scale, self.absmax_f32) if t is not None)
+
+
+def qlora_nf4_sizes(rows: int, cols: int, double_quant: bool = True) -> tuple[int, int, int]:
+    c, a, g = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().qlora_nf4_sizes(rows, cols, int(double_quant), ctypes.byref(c), ctypes.byref(a),
+                                 ctypes.byref(g)), "qlora_nf4_sizes")
+    return c.value, a.value, g.value
+
+
+def qlora_nf4_codebook() -> list[float]:
+    out = (ctypes.c_float * 16)()
+    lib().qlora_nf4_codebook(out)
+    return list(out)
+
+
+def qlora_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return int(lib().qlora_workspace_bytes(M, N, K, r))
+
+
+def empty_nf4(rows: int, cols: int, device, double_quant: bool = True,
+              keep_absmax_f32: bool = False) -> NF4Weight:
+    """Allocate (torch) the arrays of an NF4 weight."""
+    c, a, g = qlora_nf4_sizes(rows, cols, double_quant)
+    blocks = rows * cols // 64
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+    if double_quant:
+        q8 = torch.empty(a, dtype=torch.uint8, device=device)
+        s2 = torch.empty(g // 4, dtype=torch.float32, device=device)
+        af = torch.empty(blocks, dtype=torch.float32, device=device) if keep_absmax_f32 else None
+    else:
+        q8 = s2 = None
+        af = torch.empty(blocks, dtype=torch.float32, device=device)
+    return NF4Weight(rows, cols, double_quant, codes, q8, s2, af)
+
+
+def qlora_quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, double_quant: bool = True,
+                       d_status: torch.Tensor | None = None, stream=None) -> NF4Weight:
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [rows, cols]")
+    if W.dtype == torch.float32:
+        dt = QLORA_F32
+    elif W.dtype == torch.bfloat16:
+        dt = QLORA_BF16
+    else:
+        raise ValueError("W must be fp32 or bf16")
+    if out is None:
+        out = empty_nf4(W.shape[0], W.shape[1], W.device, double_quant)
+    cw = out.c()
+    _check(lib().qlora_quantize_nf4(_ptr(W), dt, ctypes.byref(cw), _ptr(d_status), _stream(stream)),
+           "qlora_quantize_nf4")
+    return out
+
+
+def qlora_dequantize(Wq: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((Wq.rows, Wq.cols), dtype=torch.bfloat16, device=Wq.codes.device)
+    cw = Wq.c()
+    _check(lib().qlora_dequantize(ctypes.byref(cw), _ptr(out), _stream(stream)), "qlora_dequantize")
+    return out
+
+
+def qlora_linear_fwd(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                     Y: torch.Tensor | None = None, T_save: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, d_status: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    M = X.shape[0]
+    r = A.shape[0]
+    if Y is None:
+        Y = torch.empty((M, Wq.rows), dtype=torch.bfloat16, device=X.device)
+    need = qlora_workspace_bytes(M, Wq.rows, Wq.cols, r)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
+    cw = Wq.c()
+    _check(lib().qlora_linear_fwd(_ptr(X), M, ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha),
+                                  _ptr(Y), _ptr(T_save), _ptr(workspace), workspace.numel(),
+                                  _ptr(d_status), _stream(stream)), "qlora_linear_fwd")
+    return Y
+
+
+def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor,
+                     B: torch.Tensor, alpha: float, T_saved: torch.Tensor | None = None,
+                     dX: torch.Tensor | None = None, dA: torch.Tensor | None = None,
+                     dB: torch.Tensor | None = None, grad_dtype=torch.float32, want_dX: bool = True,
+                     workspace: torch.Tensor | None = None, d_status: torch.Tensor | None = None,
+                     stream=None):
+    M = X.shape[0]
+    r = A.shape[0]
+    dev = X.device
+    if want_dX and dX is None:
+        dX = torch.empty((M, Wq.cols), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((r, Wq.cols), dtype=grad_dtype, device=dev)
+    if dB is None:
+        dB = torch.empty((Wq.rows, r), dtype=grad_dtype, device=dev)
+    gdt = QLORA_F32 if dA.dtype == torch.float32 else QLORA_BF16
+    need = qlora_workspace_bytes(M, Wq.rows, Wq.cols, r)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    cw = Wq.c()
+    _check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(cw), _ptr(A), _ptr(B), r,
+                                  float(alpha), _ptr(T_saved), _ptr(dX) if want_dX else None,
+                                  _ptr(dA), _ptr(dB), gdt, _ptr(workspace), workspace.numel(),
+                                  _ptr(d_status), _stream(stream)), "qlora_linear_bwd")
+    return dX, dA, dB

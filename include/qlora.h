@@ -1,0 +1,178 @@
+/*
+ * qlora.h -- C ABI of libqlora: the QLoRA frozen-base linear layer on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The frozen base weight W [rows = N out-features, cols = K in-features] is
+ * stored as blockwise NF4: 64 consecutive weights of a row share one absmax
+ * scale, each weight is the 4-bit index of the nearest of 16 normal-quantile
+ * levels, and the block scales are themselves quantised to 8 bits in groups
+ * of 256 ("QLoRA", learning-llms.pages.dev/topics/qlora, the bullets on
+ * 64-weight blocks and on NF4; "QLoRA", infra.bea.ai, §1 "How QLoRA Works",
+ * subsections "Key Innovation: NF4" and "Double Quantization").  The
+ * weight is dequantised to bf16 just in time for each matmul and never
+ * updated; the rank-r LoRA adapters A [r, K] and B [N, r] stay in bf16 and
+ * are the only tensors that receive gradients (learning-llms page, the bullet
+ * on 4-bit storage with bf16 compute, and the forward equation; infra.bea.ai
+ * page, section "The Backward Pass Through Quantization").
+ *
+ * Conventions shared by every call
+ *   - All matrices are row-major.  Activations X [M, K], Y [M, N], dY [M, N],
+ *     dX [M, K]; adapters A [r, K], B [N, r]; s = alpha / r.
+ *   - Array arguments are DEVICE pointers owned by the caller, except where a
+ *     comment says host.  bf16 arrays are passed as void*.  Every device
+ *     pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Arguments are validated synchronously; the work is enqueued
+ *     asynchronously on `stream`.  No call allocates memory, synchronises, or
+ *     keeps state between calls.
+ *   - `d_status` (nullable) is a device int the kernels OR error bits into:
+ *     QLORA_DEV_NONFINITE_BIT (non-finite weight seen by the quantiser) and
+ *     QLORA_DEV_TIMEOUT_BIT (a pipeline wait gave up after ~2 s; the kernel
+ *     then returns early and its outputs are unspecified).  The caller zeroes
+ *     it and reads it after synchronising.
+ *   - Errors: a call that returns anything but QLORA_OK has enqueued nothing.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1, /* null pointer, bad shape, misalignment, bad enum */
+  QLORA_ERR_UNSUPPORTED = 2, /* well-formed but outside what is built (e.g. block != 64) */
+  QLORA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, tensor map) */
+  QLORA_ERR_NONFINITE = 4,   /* reserved for callers mapping QLORA_DEV_NONFINITE_BIT */
+  QLORA_ERR_TIMEOUT = 5,     /* reserved for callers mapping QLORA_DEV_TIMEOUT_BIT */
+  QLORA_ERR_WORKSPACE = 6    /* workspace null or smaller than qlora_workspace_bytes() */
+} qlora_status;
+
+#define QLORA_DEV_NONFINITE_BIT 1
+#define QLORA_DEV_TIMEOUT_BIT 2
+
+typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
+
+/*
+ * One NF4 weight.  Describes caller-owned device arrays; the library never
+ * frees them.
+ *   codes       [rows, cols/2] uint8: byte j of a row holds the code of element
+ *               2j in its low nibble and of element 2j+1 in its high nibble.
+ *   absmax_q8   [rows*cols/64] uint8 (double_quant = 1): block b is elements
+ *               64b .. 64b+63 of the row-major matrix.
+ *   group_scale [ceil(rows*cols/64/256)] fp32 (double_quant = 1): group g
+ *               covers blocks 256g .. 256g+255, so groups may cross rows.
+ *   absmax_f32  [rows*cols/64] fp32 (double_quant = 0, or an optional extra
+ *               output of the quantiser when non-null).
+ * Block scale: double_quant ? float(absmax_q8[b]) * group_scale[b/256]
+ *                           : absmax_f32[b].
+ */
+typedef struct {
+  int64_t rows;          /* N */
+  int64_t cols;          /* K, a multiple of 64 */
+  int32_t blocksize;     /* must be 64 */
+  int32_t group;         /* must be 256 */
+  int32_t double_quant;  /* 1: absmax_q8 + group_scale; 0: absmax_f32 */
+  int32_t reserved;      /* must be 0 */
+  uint8_t* codes;
+  uint8_t* absmax_q8;
+  float* group_scale;
+  float* absmax_f32;
+} qlora_nf4_weight;
+
+/*
+ * Byte sizes of the three arrays of an NF4 weight: codes rows*cols/2,
+ * absmax rows*cols/64 (x4 without double quantisation), group scales
+ * 4*ceil(rows*cols/16384) (0 without).  Storage: 4 + 8/64 + 32/16384 =
+ * 4.127 bits per weight with double quantisation, 4.5 without -- the
+ * overhead figures of the learning-llms page (the bullet on 64-weight blocks
+ * and the paragraph after its memory table).
+ * Host-only; no GPU needed.  Output pointers are host pointers.
+ */
+qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int double_quant,
+                             size_t* codes_bytes, size_t* absmax_bytes,
+                             size_t* group_bytes);
+
+/*
+ * The 16 NF4 levels (code 0..15, ascending, code 7 = 0) into host out[16].
+ * Normal quantiles normalised to [-1, 1] (QLoRA paper construction).
+ */
+void qlora_nf4_codebook(float* out16);
+
+/*
+ * One-shot quantiser, run once when the model is loaded (katajob.com page,
+ * section "The mechanism": the base is quantised a single time, at load).  W: device [rows, cols], fp32 (w_dtype = QLORA_F32) or bf16.
+ * Per 64-block: absmax; x = w * fp32(1/absmax); code = nearest NF4 level
+ * (ties to the lower code); a block with absmax below FLT_MIN is all code 7.
+ * With double_quant, per 256-block group: s = fp32(max absmax / 255),
+ * q8 = min(255, rint(absmax / s)) (s = 0 and q8 = 0 when the group max is
+ * below FLT_MIN); the codes use the fp32 absmax.  out->absmax_f32 is
+ * written when non-null.  A non-finite weight sets QLORA_DEV_NONFINITE_BIT;
+ * the outputs are then unspecified.
+ */
+qlora_status qlora_quantize_nf4(const void* W, qlora_dtype w_dtype,
+                                const qlora_nf4_weight* out, int* d_status,
+                                void* stream);
+
+/*
+ * Dequantise to bf16: W_out[e] = bf16_rne(fp32(level[code] * scale)), the
+ * just-in-time bf16 reconstruction of the learning-llms page (the bullet on
+ * 4-bit storage with bf16 compute).  W_out: device [rows, cols] bf16.
+ */
+qlora_status qlora_dequantize(const qlora_nf4_weight* Wq, void* W_out, void* stream);
+
+/*
+ * Workspace bytes that qlora_linear_fwd / qlora_linear_bwd need for this
+ * shape (M tokens, weight N x K, rank r).  Host-only.  Returns 0 for an
+ * invalid shape.
+ */
+size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+
+/*
+ * Forward ("QLoRA", learning-llms page, the forward equation
+ * h = W^x + (alpha/r) B(Ax), W^ = dequant(W_4bit)), row-major:
+ *     T = X A^T  [M, r]          Y = X W^T + s T B^T  [M, N]
+ * X bf16 [M, K]; A bf16 [r, K]; B bf16 [N, r]; Y bf16 [M, N] (written).
+ * T_save (nullable) fp32 [M, r]: T for the backward.  1 <= r <= 256.
+ * W^ is dequantised tile by tile in shared memory inside the GEMM; the
+ * adapter product enters the same fp32 accumulator, one bf16 rounding per
+ * output.  Requires N % 8 == 0, K % 64 == 0.
+ */
+qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* Wq,
+                              const void* A, const void* B, int r, float alpha,
+                              void* Y, float* T_save, void* workspace,
+                              size_t ws_bytes, int* d_status, void* stream);
+
+/*
+ * Backward through the frozen base ("QLoRA", infra.bea.ai, "The Backward
+ * Pass Through Quantization": dequantise on the fly, only the adapters get
+ * gradients, the NF4 base stays frozen):
+ *     G  = dY B  [M, r]
+ *     dX = dY W^ + s G A  [M, K]      (skipped when dX is NULL)
+ *     dA = s G^T X        [r, K]
+ *     dB = s dY^T T       [N, r]
+ * dY bf16 [M, N]; X bf16 [M, K]; T_saved fp32 [M, r] from the forward, or
+ * NULL to recompute T = X A^T.  dA, dB in grad_dtype (fp32 or bf16),
+ * overwritten.  Wq is read only.  Same shape rules as the forward.
+ */
+qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M,
+                              const qlora_nf4_weight* Wq, const void* A,
+                              const void* B, int r, float alpha,
+                              const float* T_saved, void* dX, void* dA, void* dB,
+                              qlora_dtype grad_dtype, void* workspace,
+                              size_t ws_bytes, int* d_status, void* stream);
+
+/* Static string for a status code. */
+const char* qlora_status_string(qlora_status s);
+
+/* Library version, "major.minor.patch". */
+const char* qlora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_H */

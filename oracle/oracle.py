@@ -13,9 +13,9 @@ activations X [M, K], W [N, K], A [r, K], B [N, r] and s = alpha / r:
     T  = X A^T                       [M, r]
     Y  = X W^T + s T B^T             [M, N]
 
-Backward ("QLoRA", infra.bea.ai, "The Backward Pass Through Quantization":
-gradients flow through the dequantised frozen base, only the adapters get
-gradients, the NF4 base is never updated):
+Backward ("QLoRA", infra.bea.ai, section "The Backward Pass Through
+Quantization": the gradient passes through the dequantised frozen base;
+only the adapters get gradients; the NF4 base is never updated):
 
     G  = dY B                        [M, r]
     dX = dY W^ + s G A               [M, K]

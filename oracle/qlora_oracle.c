@@ -11,19 +11,18 @@
  * Every step follows the pages in their order, written as scalar loops:
  *
  *   - absmax quantiser, scale = absmax / 7, q = round(w / scale), w^ = q*scale
- *     ("QLoRA", learning-llms.pages.dev/topics/qlora: the equation under
- *     "Quantization here is just controlled rounding", and the 8-weight
- *     worked block that follows it);
+ *     ("QLoRA", learning-llms.pages.dev/topics/qlora: the absmax equation and
+ *     the 8-weight worked block that follows it);
  *   - 64-weight blocks with one absmax each, scales double-quantised to
- *     8 bits (same page, bullet "Small blocks (64 weights each)"; "QLoRA",
- *     infra.bea.ai, §1 "Double Quantization");
+ *     8 bits (same page, the bullet on 64-weight blocks; "QLoRA", infra.bea.ai,
+ *     §1 subsection "Double Quantization");
  *   - each weight stored as the index of the nearest of the 16 NF4 levels
- *     (learning-llms page, "store each weight as the index of its nearest
- *     grid point"; bullet "NF4 instead of a uniform grid");
- *   - two 4-bit codes per byte ("8 half-byte integers + one shared scale",
- *     learning-llms page, below the worked-block table);
- *   - dequantisation to bf16 for the matmul (learning-llms page, bullet
- *     "Compute never happens in 4-bit").
+ *     (learning-llms page, the sentence before the absmax equation and the
+ *     bullet on NF4);
+ *   - two 4-bit codes per byte (learning-llms page, the sentence below the
+ *     worked-block table: eight weights become eight half-bytes and a scale);
+ *   - dequantisation to bf16 for the matmul (learning-llms page, the bullet on
+ *     4-bit storage with bf16 compute).
  *
  * Readings taken where the pages are silent (each one is listed with its
  * reason in the design notes):
@@ -92,9 +91,8 @@ void oracle_bf16_to_f32(const uint16_t* in, int64_t n, float* out)
 }
 
 /* -------------------------------------------- symmetric absmax integer grid
- * learning-llms page, equation under "Quantization here is just controlled
- * rounding": scale = absmax / 7, q = round(w / scale), w^ = q * scale, for a
- * 4-bit grid; its listing clamps q to [-8, 7].  Generalised to b bits:
+ * learning-llms page, the absmax equation: scale = absmax / 7, q = round(w / scale), w^ = q * scale, for a
+ * 4-bit grid; the page's listing clamps q to [-8, 7].  Generalised to b bits:
  * scale = absmax / (2^(b-1) - 1), q clamped to [-2^(b-1), 2^(b-1) - 1].
  * round() is round-half-to-even (the listing's torch.round).
  * Returns the scale; q and w_hat are written for all n weights.
@@ -178,8 +176,8 @@ int oracle_nf4_quantize(const float* w, int64_t rows, int64_t cols,
     if (rows < 1 || cols < 1 || cols % BLOCK != 0) return ORACLE_INVALID;
     const int64_t blocks = rows * cols / BLOCK;
 
-    /* Step 1: block absmax (learning-llms page: "find its largest absolute
-       value (the absmax)"; blocks of 64 per the "Small blocks" bullet). */
+    /* Step 1: block absmax, the largest magnitude in each 64-weight block
+       (learning-llms page, absmax equation; the bullet on 64-weight blocks). */
     for (int64_t b = 0; b < blocks; ++b) {
         float m = 0.0f;
         for (int i = 0; i < BLOCK; ++i) {
