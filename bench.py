@@ -1,0 +1,546 @@
+"""Benchmark of the QLoRA NF4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one training pass of a LLaMA-7B-shaped decoder layer's seven NF4
+projections (q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008) at 2048
+tokens (batch 4 x seq 512), LoRA r=16, alpha=32: the forward of every
+projection (T = X A^T, fused dequant GEMM with the adapter folded in) and the
+backward in reverse order (G, fused dX GEMM, dA, dB).  The weights are
+quantised once before timing (the pages quantise at load time); the
+quantiser, the standalone dequantiser and the decode-shaped forward (70B MLP
+weights, M in {1, 4, 16}) are timed as separate sub-measurements of the same
+run and reported in the same JSON line.
+
+Metric: algorithmic TFLOP/s = sum over projections of 4*M*N*K + 6*M*r*(N+K)
+per step / device time.  Inputs are synthetic (seeded normal draws).
+Data-parallel over N GPUs: every rank runs the same per-GPU workload on its
+own token shard (weak scaling) and the adapter gradients dA, dB are summed
+over ranks with one NCCL all-reduce per step.
+
+--impl reference times the CPU oracle (binary64 numpy + plain C), as it
+stands, on a bounded sample of the same step (a slice of the tokens).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from bit_nf4_quantized_21_b200 import inputs  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s; NF4 GEMV weight GB/s; % of roofline"
+WL = inputs.LLAMA7B
+L2_BYTES = 126 * 1024 * 1024
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def step_flops(wl=WL, M=None) -> float:
+    M = wl.M if M is None else M
+    return float(sum(4 * M * N * K + 6 * M * wl.r * (N + K) for _, N, K in wl.shapes))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                clk, cmax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            mx = max(mx, cmax)
+            sm.append(clk)
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        busy = [c for c in sm if c > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- our path
+class Layer:
+    """Seven NF4 projections of one layer, resident on the device."""
+
+    def __init__(self, q, wl, M, device, rank):
+        self.q = q
+        self.wl = wl
+        self.M = M
+        self.proj = []
+        for i, (name, N, K) in enumerate(wl.shapes):
+            seed = inputs.matrix_seed(wl.base_seed, rank, i)
+            W = inputs.weight((N, K), wl.w_std, seed, device=device)
+            Wq = q.empty_nf4(N, K, device)
+            p = dict(name=name, N=N, K=K, W_bf16_bytes=W.numel() * 2)
+            p["Wq"] = Wq
+            p["W_tmp"] = W
+            p["X"] = inputs.normal((M, K), 1.0, seed * 16 + 1, device)
+            p["dY"] = inputs.normal((M, N), 1.0, seed * 16 + 2, device)
+            p["A"] = inputs.normal((wl.r, K), 0.01, seed * 16 + 3, device)
+            p["B"] = inputs.normal((N, wl.r), 0.01, seed * 16 + 4, device)
+            p["Y"] = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            p["T"] = torch.empty((M, wl.r), dtype=torch.float32, device=device)
+            p["dX"] = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+            p["dA"] = torch.empty((wl.r, K), dtype=torch.float32, device=device)
+            p["dB"] = torch.empty((N, wl.r), dtype=torch.float32, device=device)
+            self.proj.append(p)
+        ws = max(q.qlora_workspace_bytes(M, p["N"], p["K"], wl.r) for p in self.proj)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        # flat gradient buffer for the data-parallel all-reduce
+        self.grad_numel = sum(p["dA"].numel() + p["dB"].numel() for p in self.proj)
+
+    def quantize_all(self, events=None):
+        for p in self.proj:
+            if events is not None:
+                events.append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+                events[-1][0].record()
+            self.q.qlora_quantize_nf4(p["W_tmp"], out=p["Wq"], d_status=self.status)
+            if events is not None:
+                events[-1][1].record()
+
+    def drop_source_weights(self):
+        for p in self.proj:
+            p.pop("W_tmp", None)
+
+    def step(self, gemm_events=None):
+        """Forward of all 7 projections, then backward in reverse order."""
+        alpha = self.wl.alpha
+        for p in self.proj:
+            ev = gemm_events.pop(0) if gemm_events else None
+            self.q.qlora_linear_fwd(p["X"], p["Wq"], p["A"], p["B"], alpha, Y=p["Y"], T_save=p["T"],
+                                    workspace=self.ws, d_status=self.status, gemm_events=ev)
+        for p in reversed(self.proj):
+            ev = gemm_events.pop(0) if gemm_events else None
+            self.q.qlora_linear_bwd(p["dY"], p["X"], p["Wq"], p["A"], p["B"], alpha, T_saved=p["T"],
+                                    dX=p["dX"], dA=p["dA"], dB=p["dB"], workspace=self.ws,
+                                    d_status=self.status, gemm_events=ev)
+
+    def gemm_flops(self):
+        """Algorithmic flops of each fused-GEMM launch, in step order."""
+        r = self.wl.r
+        f = [2 * self.M * p["N"] * p["K"] + 2 * self.M * r * p["N"] for p in self.proj]
+        b = [2 * self.M * p["N"] * p["K"] + 2 * self.M * r * p["K"] for p in reversed(self.proj)]
+        return f + b
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def launches_per_step(wl) -> int:
+    # forward: T skinny + finish + GEMM; backward: G skinny + finish + dX GEMM +
+    # T split + dA skinny + finish + dB skinny + finish (+1 pad each when r % 8)
+    pad = 1 if wl.r % 8 else 0
+    return len(wl.shapes) * (3 + 8 + 2 * pad)
+
+
+def run_ours(args):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import bit_nf4_quantized_21_b200 as q
+    q.lib()  # fails loudly when the library is missing
+    peaks, peaks_src = load_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- setup: draw and quantise the layer (quantiser timed here)
+    layer = Layer(q, WL, WL.M, dev, rank)
+    torch.cuda.synchronize()
+    qev = []
+    layer.quantize_all(events=qev)
+    torch.cuda.synchronize()
+    quant_ms = sum(a.elapsed_time(b) for a, b in qev)
+    n_params = sum(p["N"] * p["K"] for p in layer.proj)
+    quant_bytes = sum(p["W_bf16_bytes"] + p["Wq"].nbytes() for p in layer.proj)
+    layer.drop_source_weights()
+    torch.cuda.empty_cache()
+    assert layer.status.item() == 0, "quantiser reported non-finite weights"
+
+    l2buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    grad_flat = torch.empty(layer.grad_numel, dtype=torch.float32, device=dev)
+
+    def allreduce_grads():
+        if world == 1:
+            return
+        off = 0
+        for p in layer.proj:
+            for t in (p["dA"], p["dB"]):
+                grad_flat[off:off + t.numel()].copy_(t.view(-1))
+                off += t.numel()
+        dist.all_reduce(grad_flat)
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        layer.step()
+        allreduce_grads()
+    torch.cuda.synchronize()
+
+    # ---- timed device steps (inputs resident), L2 flushed between steps
+    nproj = len(layer.proj)
+    gemm_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(2 * nproj)] for _ in range(args.steps)]
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush_l2(l2buf)
+        step_ev[i][0].record()
+        layer.step(gemm_events=list(gemm_ev[i]))
+        allreduce_grads()
+        step_ev[i][1].record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    gemm_ms = [[a.elapsed_time(b) for a, b in evs] for evs in gemm_ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    assert layer.status.item() == 0, f"device status {layer.status.item()}"
+    flops = step_flops() * args.steps * world
+    value = flops / (total_ms * 1e-3) / 1e12
+
+    # ---- roofline of the dominant kernel (fused NF4 GEMM), from the live events
+    gflops = layer.gemm_flops()
+    g_time = sum(sum(x) for x in gemm_ms) * 1e-3
+    g_launches = len(gflops) * args.steps
+    g_achieved = sum(gflops) * args.steps / g_time / 1e12
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    peak_burst = float(peaks.get("bf16_tflops"))
+    gemm_share = g_time * 1e3 / sum(step_ms)
+
+    # ---- end to end through host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hostX = [p["X"].cpu().pin_memory() for p in layer.proj]
+        hostdY = [p["dY"].cpu().pin_memory() for p in layer.proj]
+        hostdA = [torch.empty_like(p["dA"], device="cpu").pin_memory() for p in layer.proj]
+        hostdB = [torch.empty_like(p["dB"], device="cpu").pin_memory() for p in layer.proj]
+        h2d = sum(t.numel() * t.element_size() for t in hostX + hostdY)
+        d2h = sum(t.numel() * t.element_size() for t in hostdA + hostdB)
+        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush_l2(l2buf)
+            e_ev[i][0].record()
+            for p, hx, hdy in zip(layer.proj, hostX, hostdY):
+                p["X"].copy_(hx, non_blocking=True)
+                p["dY"].copy_(hdy, non_blocking=True)
+            layer.step()
+            allreduce_grads()
+            for p, ha, hb in zip(layer.proj, hostdA, hostdB):
+                ha.copy_(p["dA"], non_blocking=True)
+                hb.copy_(p["dB"], non_blocking=True)
+            e_ev[i][1].record()
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = sum(a.elapsed_time(b) for a, b in e_ev)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": round(flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(e_ms / args.steps, 4)}
+
+    # ---- sub-measurements: standalone dequantiser and decode-shaped forward
+    sub = {}
+    if not args.no_sub and rank == 0:
+        sub = sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_params)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(layer, args.cpu_tokens)
+
+    hbm = float(peaks["hbm_gbs"])
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "llama7b-layer-7proj-fwd+bwd", "tokens_per_gpu": WL.M,
+                   "batch": 4, "seq_len": 512, "lora_r": WL.r, "lora_alpha": WL.alpha,
+                   "projections": [[n, N, K] for n, N, K in WL.shapes],
+                   "weights": "NF4 double-quant, block 64, group 256",
+                   "flops_per_step": step_flops(), "l2": "flushed between timed steps",
+                   "parallelism": f"dp{world}"},
+        "roofline": {"bound": "tensor", "kernel": "k_gemm_nf4 (fused NF4 dequant + tcgen05 GEMM)",
+                     "achieved": round(g_achieved, 2), "peak": round(peak_sus, 1), "unit": "TFLOP/s",
+                     "frac": round(g_achieved / peak_sus, 4),
+                     "peak_source": f"{peaks_src} bf16_tflops_sustained",
+                     "frac_of_burst_peak": round(g_achieved / peak_burst, 4),
+                     "launches": g_launches, "avg_launch_us": round(g_time / g_launches * 1e6, 2),
+                     "share_of_step": round(gemm_share, 4), "traffic": None},
+        "gpu_launches": launches_per_step(WL) * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    line.update(sub)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def time_events(fn, reps, flush=None):
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        if flush is not None:
+            flush()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_params):
+    hbm = float(peaks["hbm_gbs"])
+    out = {}
+    # quantiser (timed once at setup, 7 projections, bf16 in)
+    qgbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    out["quantize"] = {"value": round(qgbs, 1), "unit": "GB/s", "params": n_params,
+                       "ms": round(quant_ms, 4), "frac_of_hbm": round(qgbs / hbm, 4),
+                       "bytes_per_param": round(quant_bytes / n_params, 4)}
+    # standalone dequantiser on the gate projection (11008 x 4096)
+    p = layer.proj[4]
+    Wout = torch.empty((p["N"], p["K"]), dtype=torch.bfloat16, device=dev)
+    f = lambda: q.qlora_dequantize(p["Wq"], out=Wout)
+    for _ in range(3):
+        f()
+    ms = time_events(f, 10, flush=lambda: l2buf.add_(1))
+    dbytes = p["Wq"].nbytes() + Wout.numel() * 2
+    dgbs = dbytes / (statistics.median(ms) * 1e-3) / 1e9
+    out["dequantize"] = {"value": round(dgbs, 1), "unit": "GB/s", "shape": [p["N"], p["K"]],
+                         "frac_of_hbm": round(dgbs / hbm, 4)}
+    del Wout
+    # decode-shaped forward: 70B MLP weights, M in {1, 4, 16}
+    wl = inputs.DECODE
+    dec = {}
+    mats = []
+    for i, (name, N, K) in enumerate(wl.shapes):
+        seed = inputs.matrix_seed(wl.base_seed, 0, i)
+        W = inputs.weight((N, K), wl.w_std, seed, device=dev, outlier_frac=wl.outlier_frac,
+                          outlier_scale=wl.outlier_scale)
+        Wq = q.qlora_quantize_nf4(W)
+        del W
+        A = inputs.normal((wl.r, K), 0.01, seed * 16 + 3, dev)
+        B = inputs.normal((N, wl.r), 0.01, seed * 16 + 4, dev)
+        mats.append((name, N, K, Wq, A, B))
+    torch.cuda.empty_cache()
+    for M in inputs.DECODE_M:
+        res = []
+        for name, N, K, Wq, A, B in mats:
+            X = inputs.normal((M, K), 1.0, 99 + M, dev)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(q.qlora_workspace_bytes(M, N, K, wl.r), dtype=torch.uint8, device=dev)
+            fn = lambda: q.qlora_linear_fwd(X, Wq, A, B, wl.alpha, Y=Y, workspace=ws)
+            for _ in range(3):
+                fn()
+            ms = statistics.median(time_events(fn, 10, flush=lambda: l2buf.add_(1)))
+            wbytes = Wq.nbytes()
+            res.append({"matrix": [N, K], "us": round(ms * 1e3, 2),
+                        "weight_gbs": round(wbytes / (ms * 1e-3) / 1e9, 1)})
+        gbs = [r_["weight_gbs"] for r_ in res]
+        dec[f"M{M}"] = {"per_matrix": res, "weight_gbs": round(sum(gbs) / len(gbs), 1),
+                        "frac_of_hbm": round(sum(gbs) / len(gbs) / hbm, 4)}
+    out["decode_gemv"] = {"unit": "GB/s of NF4 weight (121.17 MB per matrix)", **dec,
+                          "peak_hbm_gbs": hbm}
+    return out
+
+
+# ------------------------------------------------------------ CPU oracle
+def _oracle_sample(layer_np, tokens):
+    """One oracle pass over the sample: dequantise (C) + fwd + bwd (numpy f64)."""
+    import oracle as O
+    wl = WL
+    for p in layer_np:
+        Wh = O.nf4_dequantize(p["q"])
+        O.linear_fwd(p["X"][:tokens], Wh, p["A"], p["B"], wl.alpha, wl.r)
+        O.linear_bwd(p["dY"][:tokens], p["X"][:tokens], Wh, p["A"], p["B"], wl.alpha, wl.r)
+
+
+def _layer_to_host(layer, tokens):
+    import numpy as np
+    bits = lambda t: t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    out = []
+    for p in layer.proj:
+        Wq = p["Wq"]
+        out.append({"q": {"codes": Wq.codes.cpu().numpy(), "q8": Wq.absmax_q8.cpu().numpy(),
+                          "s2": Wq.group_scale.cpu().numpy(), "absmax": None, "rows": p["N"],
+                          "cols": p["K"], "double_quant": True},
+                    "X": bits(p["X"][:tokens]), "dY": bits(p["dY"][:tokens]),
+                    "A": bits(p["A"]), "B": bits(p["B"])})
+    return out
+
+
+def _cores_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(layer, tokens):
+    host = _layer_to_host(layer, tokens)
+    t0 = time.perf_counter()
+    _oracle_sample(host, tokens)
+    dt = time.perf_counter() - t0
+    flops = step_flops(M=tokens)
+    return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": _cores_used(),
+            "kind": "oracle",
+            "sample": f"one step of the same 7 projections on {tokens} of the {WL.M} tokens: "
+                      f"C dequantise + binary64 numpy fwd/bwd, {dt:.2f} s"}
+
+
+def run_reference(args):
+    """CPU oracle arm: rank 0 only; other ranks exit without work."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle as O
+    tokens = args.cpu_tokens
+    # the same inputs, drawn on the CPU, quantised by the oracle itself
+    host = []
+    for i, (name, N, K) in enumerate(WL.shapes):
+        seed = inputs.matrix_seed(WL.base_seed, 0, i)
+        W = inputs.weight((N, K), WL.w_std, seed, dtype=torch.bfloat16)
+        bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+        host.append({"q": O.nf4_quantize(W.float().numpy()),
+                     "X": bits(inputs.normal((tokens, K), 1.0, seed * 16 + 1)),
+                     "dY": bits(inputs.normal((tokens, N), 1.0, seed * 16 + 2)),
+                     "A": bits(inputs.normal((WL.r, K), 0.01, seed * 16 + 3)),
+                     "B": bits(inputs.normal((N, WL.r), 0.01, seed * 16 + 4))})
+        del W
+    for _ in range(args.warmup):
+        _oracle_sample(host, tokens)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_sample(host, tokens)
+    dt = time.perf_counter() - t0
+    value = step_flops(M=tokens) * args.steps / dt / 1e12
+    cores = _cores_used()
+    sample = (f"each step: the 7 projections on {tokens} of the {WL.M} tokens "
+              f"(C dequantise + binary64 numpy fwd/bwd)")
+    line = {"metric": METRIC, "value": round(value, 5), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "llama7b-layer-7proj-fwd+bwd", "tokens_per_step": tokens,
+                       "lora_r": WL.r, "lora_alpha": WL.alpha},
+            "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-tokens", type=int, default=64)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sub", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # timing rule: at least 3 warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -7,9 +7,11 @@
 // W^ never exists in global memory: each 64-wide slice of the contraction is
 // dequantised from the packed codes straight into the swizzled shared-memory
 // layout the tensor core reads, used for one pipeline stage and overwritten.
-// The adapter product is r extra contraction steps of the same tcgen05
-// accumulator ([X | sT] . [W^ | B]^T), so every output is one fp32 sum
-// rounded once to bf16.
+// The adapter product is extra contraction steps of the same tcgen05
+// accumulator, with s*T carried as two bf16 terms (hi = bf16(sT),
+// lo = bf16(sT - hi)):  [X | sT_hi | sT_lo] . [W^ | B | B]^T.  Every output
+// is one fp32 sum rounded once to bf16, and the adapter term keeps ~16
+// mantissa bits of s*T.
 //
 // CTA tile: 128 activation rows x 256 output columns, contraction stage 64.
 // Warp roles (320 threads):
@@ -58,6 +60,7 @@ struct GemmArgs {
   __nv_bfloat16* out;
   int num_kt;            // contraction stages over the weight
   int lora_r16;          // adapter rank rounded up to 16 (0: no adapter)
+  int64_t lora_lo_row;   // row of the adapter operand where the lo plane starts (= M)
   int* status;
 };
 
@@ -87,7 +90,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kGemmBM;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kGemmBN;   // output-column tile origin
-  const int num_lt = (args.lora_r16 + 63) / 64;
+  const int nl1 = (args.lora_r16 + 63) / 64;   // adapter stages per plane
+  const int num_lt = 2 * nl1;                  // hi plane, then lo plane
   const int total = args.num_kt + num_lt;
 
   if (threadIdx.x == 0) {
@@ -135,14 +139,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         } else {
           const int lt = it - args.num_kt;
+          const int li = lt % nl1;
+          const int64_t arow = (lt / nl1) * args.lora_lo_row + m0;
           mbar_arrive_expect_tx(fa, kGemmABytes + kGemmWBytes);
-          tma_load_2d(smem_u32(sm.a(s)), &tm_la, fa, lt * 64, static_cast<int32_t>(m0));
+          tma_load_2d(smem_u32(sm.a(s)), &tm_la, fa, li * 64, static_cast<int32_t>(arow));
           if (MODE == kModeFwd) {
-            tma_load_2d(smem_u32(sm.w(s)), &tm_lb, fa, lt * 64, static_cast<int32_t>(n0));
+            tma_load_2d(smem_u32(sm.w(s)), &tm_lb, fa, li * 64, static_cast<int32_t>(n0));
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              tma_load_2d(smem_u32(sm.w(s)) + j * 8192, &tm_lb, fa, static_cast<int32_t>(n0) + 64 * j, lt * 64);
+              tma_load_2d(smem_u32(sm.w(s)) + j * 8192, &tm_lb, fa, static_cast<int32_t>(n0) + 64 * j, li * 64);
           }
         }
         ++issued;
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t a_base = smem_u32(sm.a(s));
         const uint32_t w_base = smem_u32(sm.w(s));
-        const int nk = (it < args.num_kt) ? 4 : min(4, (args.lora_r16 - (it - args.num_kt) * 64) / 16);
+        const int nk = (it < args.num_kt) ? 4 : min(4, (args.lora_r16 - ((it - args.num_kt) % nl1) * 64) / 16);
         for (int k = 0; k < nk; ++k) {
           const uint64_t adesc = sw128_desc(a_base + k * 32, 16, 1024);
           const uint64_t bdesc = (MODE == kModeFwd) ? sw128_desc(w_base + k * 32, 16, 1024)

@@ -194,7 +194,7 @@ Ws ws_layout(const Dims& d) {
   size_t off = 0;
   w.partial = off; off += a256(part);
   w.t32 = off; off += a256(static_cast<size_t>(d.M) * d.r * 4);
-  w.sx = off; off += a256(static_cast<size_t>(d.M) * d.r8 * 2);
+  w.sx = off; off += a256(static_cast<size_t>(2 * d.M) * d.r8 * 2);
   w.ghl = off; off += a256(static_cast<size_t>(d.M) * d.Qh * 2);
   w.thl = off; off += a256(static_cast<size_t>(d.M) * d.Qh * 2);
   w.bpad = off; off += a256(static_cast<size_t>(d.N) * d.r8 * 2);
@@ -250,13 +250,20 @@ const void* padded_B(const void* B, const Dims& d, uint8_t* ws, const Ws& L, cud
 }
 
 qlora_status launch_gemm(int mode, const CUtensorMap& tact, const CUtensorMap& tcodes, const CUtensorMap& tla,
-                         const CUtensorMap& tlb, const GemmArgs& a, cudaStream_t st) {
+                         const CUtensorMap& tlb, const GemmArgs& a, const qlora_gemm_events* ev,
+                         cudaStream_t st) {
   dim3 grid(static_cast<unsigned>(cdiv(a.out_cols, kGemmBN)), static_cast<unsigned>(cdiv(a.M, kGemmBM)));
+  if (ev && ev->gemm_start && cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_start), st) != cudaSuccess)
+    return QLORA_ERR_CUDA;
   if (mode == kModeFwd)
     k_gemm_nf4<kModeFwd><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tact, tcodes, tla, tlb, a);
   else
     k_gemm_nf4<kModeDx><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tact, tcodes, tla, tlb, a);
-  return check_launch();
+  qlora_status rc = check_launch();
+  if (rc == QLORA_OK && ev && ev->gemm_end &&
+      cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_end), st) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return rc;
 }
 
 }  // namespace
@@ -336,7 +343,7 @@ qlora_status qlora_dequantize(const qlora_nf4_weight* Wq, void* W_out, void* str
 
 qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* Wq, const void* A, const void* B,
                               int r, float alpha, void* Y, float* T_save, void* workspace, size_t ws_bytes,
-                              int* d_status, void* stream) {
+                              int* d_status, const qlora_gemm_events* events, void* stream) {
   qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes);
   if (st != QLORA_OK) return st;
   if (!X || !A || !B || !Y || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y))
@@ -363,7 +370,7 @@ qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* 
   if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 32, kGemmBN,
                 CU_TENSOR_MAP_SWIZZLE_32B))
     return QLORA_ERR_CUDA;
-  if (!bf16_map(&tla, sT, d.r8, d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
+  if (!bf16_map(&tla, sT, d.r8, 2 * d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
   if (!bf16_map(&tlb, Bp, d.r8, d.N, d.r8, 64, kGemmBN)) return QLORA_ERR_CUDA;
   GemmArgs a{};
   a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
@@ -371,14 +378,15 @@ qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* 
   a.out = static_cast<__nv_bfloat16*>(Y);
   a.num_kt = static_cast<int>(d.K / 64);
   a.lora_r16 = d.r16;
+  a.lora_lo_row = d.M;
   a.status = d_status;
-  return launch_gemm(kModeFwd, tact, tcodes, tla, tlb, a, cs);
+  return launch_gemm(kModeFwd, tact, tcodes, tla, tlb, a, events, cs);
 }
 
 qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const qlora_nf4_weight* Wq, const void* A,
                               const void* B, int r, float alpha, const float* T_saved, void* dX, void* dA, void* dB,
                               qlora_dtype grad_dtype, void* workspace, size_t ws_bytes, int* d_status,
-                              void* stream) {
+                              const qlora_gemm_events* events, void* stream) {
   qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes);
   if (st != QLORA_OK) return st;
   if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
@@ -418,7 +426,7 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
     if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 128, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B))
       return QLORA_ERR_CUDA;
-    if (!bf16_map(&tla, sG, d.r8, d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&tla, sG, d.r8, 2 * d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
     if (!bf16_map(&tlb, A, d.K, d.r, d.K, 64, 64)) return QLORA_ERR_CUDA;
     GemmArgs a{};
     a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
@@ -426,8 +434,9 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
     a.out = static_cast<__nv_bfloat16*>(dX);
     a.num_kt = static_cast<int>(cdiv(d.N, 64));
     a.lora_r16 = d.r16;
+    a.lora_lo_row = d.M;
     a.status = d_status;
-    st = launch_gemm(kModeDx, tact, tcodes, tla, tlb, a, cs);
+    st = launch_gemm(kModeDx, tact, tcodes, tla, tlb, a, events, cs);
     if (st != QLORA_OK) return st;
   }
   // 3. T (saved or recomputed) -> [T_hi | T_lo]

@@ -181,8 +181,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 // ---------------------------------------------------------------- finishing
 
 // Token-indexed results (T or G): v[m, i] = sum over splits of src.
-// Writes (each optional): f32 [M, r]; s_bf16 [M, r8] = bf16(s * v) with zero
-// padding; hl [M, Qh] = [bf16(v) | bf16(v - bf16(v))] at columns [0, r) and
+// Writes (each optional): f32 [M, r]; s_bf16 [2M, r8]: rows 0..M-1 hold
+// bf16(s*v), rows M..2M-1 the remainder bf16(s*v - bf16(s*v)), zero padded;
+// hl [M, Qh] = [bf16(v) | bf16(v - bf16(v))] at columns [0, r) and
 // [r16, r16 + r), zeros elsewhere.
 __global__ void k_finish_rows(const float* __restrict__ src, int64_t src_ld, int splits,
                               int64_t split_stride, int64_t M, int r, int r8, int r16, int Qh,
@@ -199,7 +200,12 @@ __global__ void k_finish_rows(const float* __restrict__ src, int64_t src_ld, int
       for (int sp = 0; sp < splits; ++sp) v += src[sp * split_stride + m * src_ld + i];
     }
     if (f32 && i < r) f32[m * r + i] = v;
-    if (s_bf16 && i < r8) s_bf16[m * r8 + i] = __float2bfloat16_rn(s * v);
+    if (s_bf16 && i < r8) {
+      const float sv = s * v;
+      const __nv_bfloat16 h = __float2bfloat16_rn(sv);
+      s_bf16[m * r8 + i] = h;
+      s_bf16[(M + m) * r8 + i] = __float2bfloat16_rn(sv - __bfloat162float(h));
+    }
     if (hl) {
       const __nv_bfloat16 h = __float2bfloat16_rn(v);
       hl[m * Qh + i] = h;

@@ -37,6 +37,20 @@ class QloraError(RuntimeError):
         super().__init__(f"{where}: {status_string(status)} (status {status})")
 
 
+class GemmEventsC(ctypes.Structure):
+    _fields_ = [("gemm_start", ctypes.c_void_p), ("gemm_end", ctypes.c_void_p)]
+
+
+def _events(ev):
+    """(start, end) torch.cuda.Event pair -> qlora_gemm_events, or None."""
+    if ev is None:
+        return None
+    for e in ev:
+        if not e.cuda_event:      # torch creates the CUDA event on first record
+            e.record()
+    return ctypes.byref(GemmEventsC(ev[0].cuda_event, ev[1].cuda_event))
+
+
 class NF4WeightC(ctypes.Structure):
     _fields_ = [
         ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
@@ -73,10 +87,10 @@ def lib() -> ctypes.CDLL:
             L.qlora_workspace_bytes.argtypes = [I64, I64, I64, I32]
             L.qlora_workspace_bytes.restype = ctypes.c_size_t
             L.qlora_linear_fwd.argtypes = [P, I64, ctypes.POINTER(NF4WeightC), P, P, I32, F, P, P, P,
-                                           ctypes.c_size_t, P, P]
+                                           ctypes.c_size_t, P, P, P]
             L.qlora_linear_fwd.restype = I32
             L.qlora_linear_bwd.argtypes = [P, P, I64, ctypes.POINTER(NF4WeightC), P, P, I32, F, P, P,
-                                           P, P, I32, P, ctypes.c_size_t, P, P]
+                                           P, P, I32, P, ctypes.c_size_t, P, P, P]
             L.qlora_linear_bwd.restype = I32
             L.qlora_status_string.argtypes = [I32]
             L.qlora_status_string.restype = ctypes.c_char_p
@@ -195,7 +209,7 @@ def qlora_dequantize(Wq: NF4Weight, out: torch.Tensor | None = None, stream=None
 def qlora_linear_fwd(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
                      Y: torch.Tensor | None = None, T_save: torch.Tensor | None = None,
                      workspace: torch.Tensor | None = None, d_status: torch.Tensor | None = None,
-                     stream=None) -> torch.Tensor:
+                     gemm_events=None, stream=None) -> torch.Tensor:
     M = X.shape[0]
     r = A.shape[0]
     if Y is None:
@@ -206,7 +220,8 @@ def qlora_linear_fwd(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.T
     cw = Wq.c()
     _check(lib().qlora_linear_fwd(_ptr(X), M, ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha),
                                   _ptr(Y), _ptr(T_save), _ptr(workspace), workspace.numel(),
-                                  _ptr(d_status), _stream(stream)), "qlora_linear_fwd")
+                                  _ptr(d_status), _events(gemm_events), _stream(stream)),
+           "qlora_linear_fwd")
     return Y
 
 
@@ -215,7 +230,7 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, Wq: NF4Weight, A: torch.
                      dX: torch.Tensor | None = None, dA: torch.Tensor | None = None,
                      dB: torch.Tensor | None = None, grad_dtype=torch.float32, want_dX: bool = True,
                      workspace: torch.Tensor | None = None, d_status: torch.Tensor | None = None,
-                     stream=None):
+                     gemm_events=None, stream=None):
     M = X.shape[0]
     r = A.shape[0]
     dev = X.device
@@ -233,5 +248,6 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, Wq: NF4Weight, A: torch.
     _check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(cw), _ptr(A), _ptr(B), r,
                                   float(alpha), _ptr(T_saved), _ptr(dX) if want_dX else None,
                                   _ptr(dA), _ptr(dB), gdt, _ptr(workspace), workspace.numel(),
-                                  _ptr(d_status), _stream(stream)), "qlora_linear_bwd")
+                                  _ptr(d_status), _events(gemm_events), _stream(stream)),
+           "qlora_linear_bwd")
     return dX, dA, dB

@@ -58,6 +58,18 @@ typedef enum {
 typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 
 /*
+ * Optional timing hook for qlora_linear_fwd / qlora_linear_bwd: CUDA events
+ * (cudaEvent_t passed as void*) that the call records on `stream` right
+ * before and right after its fused NF4 GEMM launch, so that a caller can
+ * time that kernel alone.  The struct and either member may be NULL; the
+ * events are owned by the caller.
+ */
+typedef struct {
+  void* gemm_start;
+  void* gemm_end;
+} qlora_gemm_events;
+
+/*
  * One NF4 weight.  Describes caller-owned device arrays; the library never
  * frees them.
  *   codes       [rows, cols/2] uint8: byte j of a row holds the code of element
@@ -145,7 +157,8 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* Wq,
                               const void* A, const void* B, int r, float alpha,
                               void* Y, float* T_save, void* workspace,
-                              size_t ws_bytes, int* d_status, void* stream);
+                              size_t ws_bytes, int* d_status,
+                              const qlora_gemm_events* events, void* stream);
 
 /*
  * Backward through the frozen base ("QLoRA", infra.bea.ai, "The Backward
@@ -164,7 +177,8 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M,
                               const void* B, int r, float alpha,
                               const float* T_saved, void* dX, void* dA, void* dB,
                               qlora_dtype grad_dtype, void* workspace,
-                              size_t ws_bytes, int* d_status, void* stream);
+                              size_t ws_bytes, int* d_status,
+                              const qlora_gemm_events* events, void* stream);
 
 /* Static string for a status code. */
 const char* qlora_status_string(qlora_status s);

@@ -103,7 +103,7 @@ def _fwd(M=16, r=8, alpha=16.0, ws=None, ws_bytes=None, **ptrs):
     p.update(ptrs)
     return q.lib().qlora_linear_fwd(p["X"], M, ctypes.byref(w), p["A"], p["B"], r, alpha, p["Y"],
                                     p["T"], FAKE if ws is None else ws,
-                                    need if ws_bytes is None else ws_bytes, None, None)
+                                    need if ws_bytes is None else ws_bytes, None, None, None)
 
 
 def test_linear_fwd_validation():
@@ -124,7 +124,7 @@ def test_linear_bwd_validation():
     need = q.qlora_workspace_bytes(16, 256, 512, 8)
     L = q.lib()
     args = [FAKE, FAKE, 16, ctypes.byref(w), FAKE, FAKE, 8, 16.0, None, FAKE, FAKE, FAKE, 0, FAKE,
-            need, None, None]
+            need, None, None, None]
     bad = list(args); bad[0] = None
     assert L.qlora_linear_bwd(*bad) == 1
     bad = list(args); bad[10] = None                 # dA
