@@ -524,6 +524,40 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_only(args):
+    """One projection's forward or backward call, repeated: the small case
+    for kernel profiles (ncu) of the fused GEMM."""
+    import bit_nf4_quantized_21_b200 as q
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    name, N, K = WL.shapes[args.proj]
+    M = args.tokens
+    seed = inputs.matrix_seed(WL.base_seed, 0, args.proj)
+    Wq = q.qlora_quantize_nf4(inputs.weight((N, K), WL.w_std, seed, device=dev))
+    X = inputs.normal((M, K), 1.0, seed * 16 + 1, dev)
+    dY = inputs.normal((M, N), 1.0, seed * 16 + 2, dev)
+    A = inputs.normal((WL.r, K), 0.01, seed * 16 + 3, dev)
+    B = inputs.normal((N, WL.r), 0.01, seed * 16 + 4, dev)
+    T = torch.empty((M, WL.r), dtype=torch.float32, device=dev)
+    ws = torch.empty(q.qlora_workspace_bytes(M, N, K, WL.r), dtype=torch.uint8, device=dev)
+    q.qlora_linear_fwd(X, Wq, A, B, WL.alpha, T_save=T, workspace=ws)
+    evs = []
+    for i in range(args.warmup + args.steps):
+        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        if args.only == "gemm-fwd":
+            q.qlora_linear_fwd(X, Wq, A, B, WL.alpha, T_save=T, workspace=ws, gemm_events=ev)
+        else:
+            q.qlora_linear_bwd(dY, X, Wq, A, B, WL.alpha, T_saved=T, workspace=ws, gemm_events=ev)
+        if i >= args.warmup:
+            evs.append(ev)
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    contraction, outc = (K, N) if args.only == "gemm-fwd" else (N, K)
+    flops = 2 * M * N * K + 2 * M * WL.r * outc
+    print(json.dumps({"only": args.only, "shape": [M, N, K], "gemm_us": round(statistics.median(ms) * 1e3, 2),
+                      "gemm_tflops": round(flops / (statistics.median(ms) * 1e-3) / 1e12, 1)}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -534,9 +568,15 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--only", choices=("gemm-fwd", "gemm-dx"), default=None,
+                    help="profile mode: repeat one projection's call (see --proj, --tokens)")
+    ap.add_argument("--proj", type=int, default=4)
+    ap.add_argument("--tokens", type=int, default=2048)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # timing rule: at least 3 warm-up steps
-    if args.impl == "reference":
+    if args.only:
+        run_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
