@@ -282,6 +282,7 @@ const char* qlora_status_string(qlora_status s) {
     case QLORA_ERR_NONFINITE: return "non-finite input";
     case QLORA_ERR_TIMEOUT: return "device wait timed out";
     case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed no-allocation scratch";
   }
   return "unknown status";
 }
@@ -481,3 +482,91 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
 }
 
 }  // extern "C"
+
+// ======================================================= no-allocation forward
+// The forward of qlora_linear_fwd with its workspace carved from a fixed
+// file-scope device array instead of a caller buffer (see qlora.h for who
+// needs this).  Host code must not hand `g_noalloc_scratch` to a kernel: in
+// host code that name is only a host-side stand-in.  The device address is
+// looked up once per device with cudaGetSymbolAddress.
+namespace {
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+qlora_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QLORA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return QLORA_OK;
+}
+
+// Forward-only carve: T partials, fp32 T, s*T planes, padded B.
+Ws noalloc_fwd_layout(const Dims& d) {
+  auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  Ws w{};
+  size_t off = 0;
+  w.partial = off; off += a256(plan_skinny(d.M, d.K, d.r16).partial_bytes);
+  w.t32 = off; off += a256(static_cast<size_t>(d.M) * d.r * 4);
+  w.sx = off; off += a256(static_cast<size_t>(2 * d.M) * d.r8 * 2);
+  w.ghl = w.thl = off;
+  w.bpad = off; off += (d.r % 8) ? a256(static_cast<size_t>(d.N) * d.r8 * 2) : 0;
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" qlora_status qlora_linear_fwd_noalloc(const void* X, int64_t M, const qlora_nf4_weight* Wq,
+                                                 const void* A, const void* B, int r, float alpha, void* Y,
+                                                 float* T_save, int* d_status, void* stream) {
+  qlora_status st = check_weight(Wq, true);
+  if (st != QLORA_OK) return st;
+  if (M < 1 || M > (int64_t(1) << 31) || r < 1 || r > 256 || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  if (Wq->rows % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (!X || !A || !B || !Y || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y))
+    return QLORA_ERR_INVALID_ARG;
+  if (T_save && !aligned16(T_save)) return QLORA_ERR_INVALID_ARG;
+  const Dims d = dims_of(M, Wq->rows, Wq->cols, r);
+  const Ws L = noalloc_fwd_layout(d);
+  if (L.total > QLORA_NOALLOC_SCRATCH_BYTES) return QLORA_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != QLORA_OK) return st;
+  if (!ensure_smem_attrs()) return QLORA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  const float s = alpha / static_cast<float>(r);
+  float* t32 = T_save ? T_save : reinterpret_cast<float*>(ws + L.t32);
+  __nv_bfloat16* sT = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
+
+  st = run_T(X, A, d, s, ws, L, t32, sT, d_status, cs);
+  if (st != QLORA_OK) return st;
+  const void* Bp = padded_B(B, d, ws, L, cs, &st);
+  if (st != QLORA_OK) return st;
+
+  CUtensorMap tact, tcodes, tla, tlb;
+  if (!bf16_map(&tact, X, d.K, d.M, d.K, 64, kGemmBM)) return QLORA_ERR_CUDA;
+  if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 32, kGemmBN,
+                CU_TENSOR_MAP_SWIZZLE_32B))
+    return QLORA_ERR_CUDA;
+  if (!bf16_map(&tla, sT, d.r8, 2 * d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
+  if (!bf16_map(&tlb, Bp, d.r8, d.N, d.r8, 64, kGemmBN)) return QLORA_ERR_CUDA;
+  GemmArgs a{};
+  a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
+  a.wN = d.N; a.wK = d.K; a.M = d.M; a.out_cols = d.N; a.ldo = d.N;
+  a.out = static_cast<__nv_bfloat16*>(Y);
+  a.num_kt = static_cast<int>(d.K / 64);
+  a.lora_r16 = d.r16;
+  a.lora_lo_row = d.M;
+  a.status = d_status;
+  return launch_gemm(kModeFwd, tact, tcodes, tla, tlb, a, nullptr, cs);
+}

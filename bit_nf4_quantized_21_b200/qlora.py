@@ -27,7 +27,7 @@ DEV_TIMEOUT = 2
 EXPORTED = (
     "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
-    "qlora_version",
+    "qlora_version", "qlora_linear_fwd_noalloc",
 )
 
 
@@ -92,6 +92,9 @@ def lib() -> ctypes.CDLL:
             L.qlora_linear_bwd.argtypes = [P, P, I64, ctypes.POINTER(NF4WeightC), P, P, I32, F, P, P,
                                            P, P, I32, P, ctypes.c_size_t, P, P, P]
             L.qlora_linear_bwd.restype = I32
+            L.qlora_linear_fwd_noalloc.argtypes = [P, I64, ctypes.POINTER(NF4WeightC), P, P, I32, F, P,
+                                                   P, P, P]
+            L.qlora_linear_fwd_noalloc.restype = I32
             L.qlora_status_string.argtypes = [I32]
             L.qlora_status_string.restype = ctypes.c_char_p
             L.qlora_version.argtypes = []
@@ -251,3 +254,21 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, Wq: NF4Weight, A: torch.
                                   _ptr(d_status), _events(gemm_events), _stream(stream)),
            "qlora_linear_bwd")
     return dX, dA, dB
+
+
+def qlora_linear_fwd_noalloc(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor,
+                             alpha: float, Y: torch.Tensor | None = None,
+                             T_save: torch.Tensor | None = None,
+                             d_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The forward with the library's fixed device scratch instead of a
+    workspace, for callers that cannot allocate device memory (see
+    qlora.h).  Allocates Y only when the caller passes none."""
+    M = X.shape[0]
+    r = A.shape[0]
+    if Y is None:
+        Y = torch.empty((M, Wq.rows), dtype=torch.bfloat16, device=X.device)
+    cw = Wq.c()
+    _check(lib().qlora_linear_fwd_noalloc(_ptr(X), M, ctypes.byref(cw), _ptr(A), _ptr(B), r,
+                                          float(alpha), _ptr(Y), _ptr(T_save), _ptr(d_status),
+                                          _stream(stream)), "qlora_linear_fwd_noalloc")
+    return Y

@@ -49,7 +49,8 @@ typedef enum {
   QLORA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, tensor map) */
   QLORA_ERR_NONFINITE = 4,   /* reserved for callers mapping QLORA_DEV_NONFINITE_BIT */
   QLORA_ERR_TIMEOUT = 5,     /* reserved for callers mapping QLORA_DEV_TIMEOUT_BIT */
-  QLORA_ERR_WORKSPACE = 6    /* workspace null or smaller than qlora_workspace_bytes() */
+  QLORA_ERR_WORKSPACE = 6,   /* workspace null or smaller than qlora_workspace_bytes() */
+  QLORA_ERR_SCRATCH_LIMIT = 7 /* problem needs more than the fixed no-allocation scratch */
 } qlora_status;
 
 #define QLORA_DEV_NONFINITE_BIT 1
@@ -179,6 +180,36 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M,
                               qlora_dtype grad_dtype, void* workspace,
                               size_t ws_bytes, int* d_status,
                               const qlora_gemm_events* events, void* stream);
+
+/*
+ * Forward without a caller workspace, for callers that cannot allocate
+ * device memory: a plugin host that hands a kernel only its input and
+ * output buffers, a process whose device memory is held by another
+ * allocator's pool, or a latency-critical loop that must not hit the
+ * implicit synchronisation a device allocation can cause.  There is no
+ * counterpart on the pages; it computes exactly what qlora_linear_fwd
+ * computes, with the same kernels.
+ *
+ * Scratch: one file-scope device array of QLORA_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) per GPU, held from library load until process exit.  A problem
+ * whose forward scratch (split-K partials of T, fp32 T, the two bf16 planes
+ * of s*T, a padded copy of B when r % 8 != 0) does not fit is rejected with
+ * QLORA_ERR_SCRATCH_LIMIT before anything is enqueued; e.g. M = 8192,
+ * r = 64 fits.  Every region is fully written before it is read, so nothing
+ * needs clearing between calls.
+ *
+ * All calls on a device share the one array: calls whose work overlaps on
+ * the GPU (different streams, or different host threads) race and give
+ * wrong results; serialise them (same stream, or events).  The first call
+ * on each device looks up the array's device address with that device
+ * current; make that first call before any stream capture.  The call itself
+ * allocates nothing (no cudaMalloc, no cudaFree, no allocating library
+ * routine).  Arguments as for qlora_linear_fwd, minus the workspace.
+ */
+#define QLORA_NOALLOC_SCRATCH_BYTES (16u << 20)
+qlora_status qlora_linear_fwd_noalloc(const void* X, int64_t M, const qlora_nf4_weight* Wq,
+                                      const void* A, const void* B, int r, float alpha,
+                                      void* Y, float* T_save, int* d_status, void* stream);
 
 /* Static string for a status code. */
 const char* qlora_status_string(qlora_status s);

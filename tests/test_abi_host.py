@@ -61,7 +61,7 @@ def test_workspace_query():
 
 
 def test_status_strings():
-    for s in range(7):
+    for s in range(8):
         assert q.status_string(s)
     assert q.status_string(0) == "ok"
 

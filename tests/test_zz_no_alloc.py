@@ -1,0 +1,78 @@
+"""The no-allocation forward (qlora_linear_fwd_noalloc), called through the
+C ABI, against the workspace forward (qlora_linear_fwd).
+
+It serves callers that cannot allocate device memory themselves (plugin
+hosts that pass only inputs and outputs, processes whose memory sits in
+another allocator's pool, loops that must not synchronise on an
+allocation); its scratch is the library's fixed 16 MiB device array, which
+keeps the previous call's contents -- hence two calls in a row with
+different inputs.  This file sorts last so that a run stopping at the first
+failure has already run every other test; it also passes on its own in a
+fresh process.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import bit_nf4_quantized_21_b200 as q
+from bit_nf4_quantized_21_b200 import inputs
+from bit_nf4_quantized_21_b200.qlora import NF4WeightC
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL = 2e-3
+
+
+def _call_noalloc(X, Wq, A, B, alpha, Y, T):
+    cw = Wq.c()
+    rc = q.lib().qlora_linear_fwd_noalloc(
+        X.data_ptr(), X.shape[0], ctypes.byref(cw), A.data_ptr(), B.data_ptr(), A.shape[0],
+        float(alpha), Y.data_ptr(), T.data_ptr() if T is not None else None, None,
+        torch.cuda.current_stream().cuda_stream)
+    return rc
+
+
+@pytest.mark.parametrize("M,N,K,r", [(200, 264, 576, 8), (2048, 4096, 4096, 16), (96, 136, 448, 5)])
+def test_noalloc_forward_matches_workspace_forward_twice(M, N, K, r):
+    alpha = 2.0 * r
+    for call, seed in enumerate((101, 202)):          # two calls in a row, different inputs
+        W = inputs.weight((N, K), 0.02, seed + M, device=DEV)
+        Wq = q.qlora_quantize_nf4(W)
+        X = inputs.normal((M, K), 1.0, seed + 1, DEV)
+        A = inputs.normal((r, K), 0.01, seed + 3, DEV)
+        B = inputs.normal((N, r), 0.01, seed + 4, DEV)
+        Y_ref = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+        T_ref = torch.empty((M, r), dtype=torch.float32, device=DEV)
+        q.qlora_linear_fwd(X, Wq, A, B, alpha, Y=Y_ref, T_save=T_ref)
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+        T = torch.full((M, r), float("nan"), dtype=torch.float32, device=DEV)
+        assert _call_noalloc(X, Wq, A, B, alpha, Y, T) == 0
+        Y2 = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+        assert _call_noalloc(X, Wq, A, B, alpha, Y2, None) == 0   # T kept in the scratch
+        torch.cuda.synchronize()
+        y_ref = Y_ref.float().cpu().numpy()
+        for got in (Y, Y2):
+            g = got.float().cpu().numpy()
+            assert np.isfinite(g).all(), f"call {call}: unwritten outputs"
+            assert O.rel_fro(g, y_ref) <= TOL
+        assert O.rel_fro(T.cpu().numpy(), T_ref.cpu().numpy()) <= 1e-6
+
+
+def test_noalloc_rejects_problems_beyond_the_scratch():
+    W = inputs.weight((256, 22016), 0.02, 7, device=DEV)
+    Wq = q.qlora_quantize_nf4(W)
+    cw = Wq.c()
+    M = 16384                                   # 64-rank forward scratch ~21 MB > 16 MiB
+    X = torch.empty((M, 22016), dtype=torch.bfloat16, device=DEV)
+    A = torch.empty((64, 22016), dtype=torch.bfloat16, device=DEV)
+    B = torch.empty((256, 64), dtype=torch.bfloat16, device=DEV)
+    Y = torch.empty((M, 256), dtype=torch.bfloat16, device=DEV)
+    rc = q.lib().qlora_linear_fwd_noalloc(X.data_ptr(), M, ctypes.byref(cw), A.data_ptr(), B.data_ptr(), 64,
+                                          16.0, Y.data_ptr(), None, None,
+                                          torch.cuda.current_stream().cuda_stream)
+    assert rc == 7 and "scratch" in q.status_string(rc)
