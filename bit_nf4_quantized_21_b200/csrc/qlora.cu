@@ -23,6 +23,7 @@
 #include "codec.cuh"
 #include "gemm_nf4.cuh"
 #include "skinny.cuh"
+#include "gemm_nf4_pair.cuh"
 
 using namespace qlora;
 
@@ -82,6 +83,8 @@ bool ensure_smem_attrs() {
   const int max_smem = 227 * 1024;
   bool ok = cudaFuncSetAttribute(k_gemm_nf4<kModeFwd>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_gemm_nf4<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeFwd>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
@@ -266,6 +269,73 @@ qlora_status launch_gemm(int mode, const CUtensorMap& tact, const CUtensorMap& t
   return rc;
 }
 
+
+// Fused NF4 GEMM of one call: tensor maps + dispatch.  M > 128 takes the
+// 2-SM pair kernel (256 x 256 tiles per pair), smaller M the 1-CTA kernel.
+//   fwd: act = X [M, K], la = s*T planes [2M, r8], lb = B [N, r8], out Y [M, N]
+//   dX : act = dY [M, N], la = s*G planes [2M, r8], lb = A [r, K], out dX [M, K]
+qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, const Dims& d, const void* la,
+                       const void* lb, void* out, const qlora_gemm_events* ev, int* status, cudaStream_t cs) {
+  const bool pair = d.M > 128;
+  const bool fwd = mode == kModeFwd;
+  CUtensorMap tact, tcodes, tla, tlb;
+  if (fwd) {
+    if (!bf16_map(&tact, act, d.K, d.M, d.K, 64, 128)) return QLORA_ERR_CUDA;
+    if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 32, pair ? 128 : kGemmBN,
+                  CU_TENSOR_MAP_SWIZZLE_32B))
+      return QLORA_ERR_CUDA;
+    if (!bf16_map(&tlb, lb, d.r8, d.N, d.r8, 64, pair ? 128 : kGemmBN)) return QLORA_ERR_CUDA;
+  } else {
+    if (!bf16_map(&tact, act, d.N, d.M, d.N, 64, 128)) return QLORA_ERR_CUDA;
+    if (pair) {
+      if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 64, 64,
+                    CU_TENSOR_MAP_SWIZZLE_64B))
+        return QLORA_ERR_CUDA;
+    } else {
+      if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 128, 64,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+        return QLORA_ERR_CUDA;
+    }
+    if (!bf16_map(&tlb, lb, d.K, d.r, d.K, 64, 64)) return QLORA_ERR_CUDA;
+  }
+  if (!bf16_map(&tla, la, d.r8, 2 * d.M, d.r8, 64, 128)) return QLORA_ERR_CUDA;
+  GemmArgs a{};
+  a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
+  a.wN = d.N; a.wK = d.K; a.M = d.M;
+  a.out_cols = fwd ? d.N : d.K;
+  a.ldo = a.out_cols;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.num_kt = static_cast<int>(fwd ? d.K / 64 : cdiv(d.N, 64));
+  a.lora_r16 = d.r16;
+  a.lora_lo_row = d.M;
+  a.status = status;
+  if (!pair) return launch_gemm(mode, tact, tcodes, tla, tlb, a, ev, cs);
+
+  if (ev && ev->gemm_start && cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_start), cs) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * cdiv(a.out_cols, 256)), static_cast<unsigned>(cdiv(d.M, 256)));
+  cfg.blockDim = dim3(kPairThreads);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cfg.stream = cs;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd>, tact, tcodes, tla, tlb, a)
+                      : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx>, tact, tcodes, tla, tlb, a);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  if (ev && ev->gemm_end && cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_end), cs) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
+
 }  // namespace
 
 // =================================================================== ABI
@@ -366,22 +436,7 @@ qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* 
   if (st != QLORA_OK) return st;
 
   // 2. Y = X W^T + (sT) B^T
-  CUtensorMap tact, tcodes, tla, tlb;
-  if (!bf16_map(&tact, X, d.K, d.M, d.K, 64, kGemmBM)) return QLORA_ERR_CUDA;
-  if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 32, kGemmBN,
-                CU_TENSOR_MAP_SWIZZLE_32B))
-    return QLORA_ERR_CUDA;
-  if (!bf16_map(&tla, sT, d.r8, 2 * d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
-  if (!bf16_map(&tlb, Bp, d.r8, d.N, d.r8, 64, kGemmBN)) return QLORA_ERR_CUDA;
-  GemmArgs a{};
-  a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
-  a.wN = d.N; a.wK = d.K; a.M = d.M; a.out_cols = d.N; a.ldo = d.N;
-  a.out = static_cast<__nv_bfloat16*>(Y);
-  a.num_kt = static_cast<int>(d.K / 64);
-  a.lora_r16 = d.r16;
-  a.lora_lo_row = d.M;
-  a.status = d_status;
-  return launch_gemm(kModeFwd, tact, tcodes, tla, tlb, a, events, cs);
+  return run_fused(kModeFwd, X, Wq, d, sT, Bp, Y, events, d_status, cs);
 }
 
 qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const qlora_nf4_weight* Wq, const void* A,
@@ -422,22 +477,7 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
   }
   // 2. dX = dY W^ + (sG) A
   if (dX) {
-    CUtensorMap tact, tcodes, tla, tlb;
-    if (!bf16_map(&tact, dY, d.N, d.M, d.N, 64, kGemmBM)) return QLORA_ERR_CUDA;
-    if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 128, 64,
-                  CU_TENSOR_MAP_SWIZZLE_128B))
-      return QLORA_ERR_CUDA;
-    if (!bf16_map(&tla, sG, d.r8, 2 * d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
-    if (!bf16_map(&tlb, A, d.K, d.r, d.K, 64, 64)) return QLORA_ERR_CUDA;
-    GemmArgs a{};
-    a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
-    a.wN = d.N; a.wK = d.K; a.M = d.M; a.out_cols = d.K; a.ldo = d.K;
-    a.out = static_cast<__nv_bfloat16*>(dX);
-    a.num_kt = static_cast<int>(cdiv(d.N, 64));
-    a.lora_r16 = d.r16;
-    a.lora_lo_row = d.M;
-    a.status = d_status;
-    st = launch_gemm(kModeDx, tact, tcodes, tla, tlb, a, events, cs);
+    st = run_fused(kModeDx, dY, Wq, d, sG, A, dX, events, d_status, cs);
     if (st != QLORA_OK) return st;
   }
   // 3. T (saved or recomputed) -> [T_hi | T_lo]
@@ -553,20 +593,5 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const void* X, int64_t M, const
   const void* Bp = padded_B(B, d, ws, L, cs, &st);
   if (st != QLORA_OK) return st;
 
-  CUtensorMap tact, tcodes, tla, tlb;
-  if (!bf16_map(&tact, X, d.K, d.M, d.K, 64, kGemmBM)) return QLORA_ERR_CUDA;
-  if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 32, kGemmBN,
-                CU_TENSOR_MAP_SWIZZLE_32B))
-    return QLORA_ERR_CUDA;
-  if (!bf16_map(&tla, sT, d.r8, 2 * d.M, d.r8, 64, kGemmBM)) return QLORA_ERR_CUDA;
-  if (!bf16_map(&tlb, Bp, d.r8, d.N, d.r8, 64, kGemmBN)) return QLORA_ERR_CUDA;
-  GemmArgs a{};
-  a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
-  a.wN = d.N; a.wK = d.K; a.M = d.M; a.out_cols = d.N; a.ldo = d.N;
-  a.out = static_cast<__nv_bfloat16*>(Y);
-  a.num_kt = static_cast<int>(d.K / 64);
-  a.lora_r16 = d.r16;
-  a.lora_lo_row = d.M;
-  a.status = d_status;
-  return launch_gemm(kModeFwd, tact, tcodes, tla, tlb, a, nullptr, cs);
+  return run_fused(kModeFwd, X, Wq, d, sT, Bp, Y, nullptr, d_status, cs);
 }
