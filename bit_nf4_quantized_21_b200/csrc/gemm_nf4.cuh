@@ -214,7 +214,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int s = it % kGemmStages;
       const float scale = scale_next;
       const bool valid = (wn < args.wN) && (kb < KB);
-      if (it + 1 < args.num_kt) scale_next = scale_of(wn + wn_step, kb + kb_step);
       if (!mbar_wait(smem_u32(&full_a[s]), (it / kGemmStages) & 1, abort_flag, args.status)) break;
       if (it < args.num_kt) {
         uint8_t* wdst = sm.w(s) + wrow_off;
@@ -248,6 +247,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         fence_proxy_async_smem();
       }
       mbar_arrive(smem_u32(&full_b[s]));
+      // next stage's scale, loaded after the arrive so its release does not wait on it
+      if (it + 1 < args.num_kt) scale_next = scale_of(wn + wn_step, kb + kb_step);
       wn += wn_step;
       kb += kb_step;
     }

@@ -9,17 +9,26 @@
 //   half), weight rows (forward) or output columns (dX) n0 + 128r .. +127
 //   (MMA B half), and TMEM rows for its 128 activation rows x 256 columns.
 //
-// Pipeline per 64-deep stage (6-stage ring):
-//   - each CTA's producer loads its packed codes with a local TMA (local
-//     barrier full_c) and its activation tile with a pair TMA whose bytes
-//     complete on the leader's barrier full_a (the leader sets expect-tx for
-//     both CTAs);
-//   - one of two dequant warp groups (stages alternate between them) turns
-//     the codes into the bf16 B half, fences it for the async proxy and
-//     arrives (one arrive per warp) on the leader's barrier full_b;
-//   - the leader's MMA thread waits full_a and full_b, issues 4
-//     tcgen05.mma.cta_group::2 (M 256, N 256, K 16) and commits to `empty`
-//     in both CTAs (multicast commit).
+// Three shared-memory rings per CTA; stage `it` (64 deep) uses slot
+// it % depth of each:
+//   activations  5 x 16 KB  pair TMA by producer lane 0, completing on the
+//                           leader's full_a; freed by the MMA (empty_a)
+//   codes        8 x  4 KB  local TMA by producer lane 1 (full_c); freed by
+//                           the dequant warps once the codes are in
+//                           registers (empty_c)
+//   bf16 weight  6 x 16 KB  written by dequant group it % 3 after the MMA
+//                           freed the slot (empty_w); one arrive per warp
+//                           on the leader's full_w
+// Ring depths follow measured hand-off latencies: every hop (commit ->
+// barrier -> wake -> load or decode -> arrive -> wake) costs hundreds of
+// cycles, and the decode loop has the most hops, so the weight ring is the
+// deepest of the 16 KB rings.  The leader's
+// MMA thread waits full_a and full_w, issues 4 tcgen05.mma.cta_group::2
+// (M 256, N 256, K 16) and commits to empty_a and empty_w in both CTAs
+// (multicast commits).  Adapter stages load their B operand by TMA into the
+// weight slot, issued by the dequant group that owns the slot.
+// Every waiter waits for each phase of a barrier in order (no waiter can be
+// two phases behind), which is what makes the 1-bit phase parity safe.
 // Epilogue: every CTA reads its own TMEM half (tcgen05.ld) and writes bf16.
 #pragma once
 #include "nf4_decode.cuh"
@@ -27,15 +36,22 @@
 
 namespace qlora {
 
-constexpr int kPairStages = 6;
-constexpr int kPairThreads = 320;
+constexpr int kPairRingA = 5;                    // activation ring depth
+constexpr int kPairRingC = 8;                    // packed-code ring depth
+constexpr int kPairRingW = 6;                    // dequantised-weight ring depth
+constexpr int kPairDeqGroups = 3;                // group it % 3 decodes stage it (owns W slots g, g + 3)
+static_assert(kPairRingW % kPairDeqGroups == 0, "each weight slot must belong to one dequant group");
+constexpr int kPairDeqWarps = 4;                 // warps per group (128 weight rows)
+constexpr int kPairThreads = 64 + kPairDeqGroups * kPairDeqWarps * 32;
 constexpr uint32_t kPairABytes = 128 * 64 * 2;   // 16 KB activations (this CTA's half)
 constexpr uint32_t kPairWBytes = 128 * 64 * 2;   // 16 KB dequantised weight half
 constexpr uint32_t kPairCBytes = 128 * 64 / 2;   //  4 KB packed codes
-constexpr uint32_t kPairStageBytes = kPairABytes + kPairWBytes + kPairCBytes;
-constexpr uint32_t kPairSmemBytes = kPairStages * kPairStageBytes + 1024 + 512;
+constexpr uint32_t kPairOffW = kPairRingA * kPairABytes;
+constexpr uint32_t kPairOffC = kPairOffW + kPairRingW * kPairWBytes;
+constexpr uint32_t kPairOffBar = kPairOffC + kPairRingC * kPairCBytes;
+constexpr uint32_t kPairSmemBytes = kPairOffBar + 1024 /*align*/ + 512 /*bars*/ + 4 * kPairDeqGroups * 128;
 constexpr uint32_t kPairTmemCols = 256;
-constexpr int kPairDeqWarps = 4;                 // per stage, per CTA
+static_assert(kPairSmemBytes <= 227 * 1024, "pair kernel shared memory");
 
 template <int MODE>
 __global__ void __launch_bounds__(kPairThreads, 1)
@@ -44,17 +60,22 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  auto slot_a = [&](int s) { return base + s * kPairStageBytes; };
-  auto slot_w = [&](int s) { return base + s * kPairStageBytes + kPairABytes; };
-  auto slot_c = [&](int s) { return base + s * kPairStageBytes + kPairABytes + kPairWBytes; };
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kPairStages * kPairStageBytes);
-  uint64_t* full_a = bars;                          // leader: both activation halves (+ adapter tiles)
-  uint64_t* full_c = bars + kPairStages;            // local: this CTA's codes
-  uint64_t* full_b = bars + 2 * kPairStages;        // leader: both dequantised halves
-  uint64_t* empty = bars + 3 * kPairStages;         // local: MMA done with the stage (multicast commit)
-  uint64_t* acc_full = bars + 4 * kPairStages;      // local: accumulator complete (multicast commit)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * kPairStages + 1);
+  auto slot_a = [&](int it) { return base + (it % kPairRingA) * kPairABytes; };
+  auto slot_w = [&](int it) { return base + kPairOffW + (it % kPairRingW) * kPairWBytes; };
+  auto slot_c = [&](int it) { return base + kPairOffC + (it % kPairRingC) * kPairCBytes; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kPairOffBar);
+  uint64_t* full_a = bars;                                  // [A] leader: activation halves (+ adapter tiles)
+  uint64_t* empty_a = full_a + kPairRingA;                  // [A] local: MMA done with the activations
+  uint64_t* full_c = empty_a + kPairRingA;                  // [C] local: codes landed
+  uint64_t* empty_c = full_c + kPairRingC;                  // [C] local: codes copied to registers
+  uint64_t* full_w = empty_c + kPairRingC;                  // [W] leader: both weight halves written
+  uint64_t* empty_w = full_w + kPairRingW;                  // [W] local: MMA done with the weights
+  uint64_t* acc_full = empty_w + kPairRingW;                // local: accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile uint32_t* dep_scratch = reinterpret_cast<volatile uint32_t*>(bars + 64);   // one word per dequant thread
+  auto par = [](int it, int depth) { return static_cast<uint32_t>((it / depth) & 1); };
+  auto prev_par = [](int it, int depth) { return static_cast<uint32_t>(((it / depth) + 1) & 1); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -67,11 +88,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int total = args.num_kt + num_lt;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPairStages; ++s) {
-      mbar_init(smem_u32(&full_a[s]), 1);
-      mbar_init(smem_u32(&full_c[s]), 1);
-      mbar_init(smem_u32(&full_b[s]), 2 * kPairDeqWarps);
-      mbar_init(smem_u32(&empty[s]), 1);
+    for (int i = 0; i < kPairRingA; ++i) { mbar_init(smem_u32(&full_a[i]), 1); mbar_init(smem_u32(&empty_a[i]), 1); }
+    for (int i = 0; i < kPairRingC; ++i) {
+      mbar_init(smem_u32(&full_c[i]), 1);
+      mbar_init(smem_u32(&empty_c[i]), kPairDeqWarps);
+    }
+    for (int i = 0; i < kPairRingW; ++i) {
+      mbar_init(smem_u32(&full_w[i]), 2 * kPairDeqWarps);
+      mbar_init(smem_u32(&empty_w[i]), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
     *abort_flag = 0;
@@ -95,48 +119,62 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // activation tiles (and, in the adapter stages, the adapter B tiles)
       int issued = 0;
       for (int it = 0; it < total; ++it) {
-        const int s = it % kPairStages;
-        if (it >= kPairStages &&
-            !mbar_wait_cluster(smem_u32(&empty[s]), ((it / kPairStages) + 1) & 1, abort_flag, args.status))
+        const int ia = it % kPairRingA;
+        if (it >= kPairRingA &&
+            !mbar_wait(smem_u32(&empty_a[ia]), prev_par(it, kPairRingA), abort_flag, args.status))
           break;
-        const uint32_t fa = leader_bar(&full_a[s]);
-        const uint32_t fc = smem_u32(&full_c[s]);
+        const uint32_t fa = leader_bar(&full_a[ia]);
         if (it < args.num_kt) {
-          mbar_arrive_expect_tx(fc, kPairCBytes);
-          if (MODE == kModeFwd)
-            tma_load_2d(smem_u32(slot_c(s)), &tm_codes, fc, it * 32, static_cast<int32_t>(nc0));
-          else
-            tma_load_2d(smem_u32(slot_c(s)), &tm_codes, fc, static_cast<int32_t>(nc0 / 2), it * 64);
-          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[s]), 2 * kPairABytes);
-          tma_load_2d_pair(smem_u32(slot_a(s)), &tm_act, fa, it * 64, static_cast<int32_t>(m0));
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * kPairABytes);
+          tma_load_2d_pair(smem_u32(slot_a(it)), &tm_act, fa, it * 64, static_cast<int32_t>(m0));
         } else {
+          // adapter stage: the A tile here; the adapter B tile is loaded into
+          // the weight slot by the dequant group that owns the slot (it waits
+          // for every phase of that slot in order; this thread runs up to a
+          // whole activation ring ahead and would alias the slot's phases)
           const int lt = it - args.num_kt;
           const int li = lt % nl1;
           const int64_t arow = (lt / nl1) * args.lora_lo_row + m0;
-          mbar_arrive(fc);   // no codes: keeps the dequant warps' phases in step
-          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[s]), 2 * (kPairABytes + kPairWBytes));
-          tma_load_2d_pair(smem_u32(slot_a(s)), &tm_la, fa, li * 64, static_cast<int32_t>(arow));
-          if (MODE == kModeFwd) {
-            tma_load_2d_pair(smem_u32(slot_w(s)), &tm_lb, fa, li * 64, static_cast<int32_t>(nc0));
-          } else {
-            tma_load_2d_pair(smem_u32(slot_w(s)), &tm_lb, fa, static_cast<int32_t>(nc0), li * 64);
-            tma_load_2d_pair(smem_u32(slot_w(s)) + 8192, &tm_lb, fa, static_cast<int32_t>(nc0) + 64, li * 64);
-          }
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * (kPairABytes + kPairWBytes));
+          tma_load_2d_pair(smem_u32(slot_a(it)), &tm_la, fa, li * 64, static_cast<int32_t>(arow));
+        }
+        ++issued;
+      }
+      if (*abort_flag && leader) {
+        for (int it = max(0, issued - kPairRingA); it < issued; ++it) {
+          const uint32_t fa = smem_u32(&full_a[it % kPairRingA]);
+          const uint64_t t1 = global_ns();
+          while (!mbar_try_wait_cluster(fa, par(it, kPairRingA)) && global_ns() - t1 < 200000000ull) {}
+        }
+      }
+    } else if (lane == 1) {
+      // packed codes, freed by the dequant warps (runs ahead of the MMA)
+      int issued = 0;
+      for (int it = 0; it < total; ++it) {
+        const int ic = it % kPairRingC;
+        if (it >= kPairRingC &&
+            !mbar_wait(smem_u32(&empty_c[ic]), prev_par(it, kPairRingC), abort_flag, args.status))
+          break;
+        const uint32_t fc = smem_u32(&full_c[ic]);
+        if (it < args.num_kt) {
+          mbar_arrive_expect_tx(fc, kPairCBytes);
+          if (MODE == kModeFwd)
+            tma_load_2d(smem_u32(slot_c(it)), &tm_codes, fc, it * 32, static_cast<int32_t>(nc0));
+          else
+            tma_load_2d(smem_u32(slot_c(it)), &tm_codes, fc, static_cast<int32_t>(nc0 / 2), it * 64);
+        } else {
+          mbar_arrive(fc);   // no codes in adapter stages: keeps the dequant warps' phases in step
         }
         ++issued;
       }
       if (*abort_flag) {
-        for (int it = max(0, issued - kPairStages); it < issued; ++it) {
-          const uint32_t fc = smem_u32(&full_c[it % kPairStages]);
+        for (int it = max(0, issued - kPairRingC); it < issued; ++it) {
+          const uint32_t fc = smem_u32(&full_c[it % kPairRingC]);
           const uint64_t t0 = global_ns();
-          while (!mbar_try_wait(fc, (it / kPairStages) & 1) && global_ns() - t0 < 200000000ull) {}
-          if (leader) {
-            const uint32_t fa = smem_u32(&full_a[it % kPairStages]);
-            const uint64_t t1 = global_ns();
-            while (!mbar_try_wait_cluster(fa, (it / kPairStages) & 1) && global_ns() - t1 < 200000000ull) {}
-          }
+          while (!mbar_try_wait(fc, par(it, kPairRingC)) && global_ns() - t0 < 200000000ull) {}
         }
       }
     }
@@ -145,13 +183,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     if (leader && lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(256, 256, 0, MODE == kModeDx ? 1 : 0);
       for (int it = 0; it < total; ++it) {
-        const int s = it % kPairStages;
-        const uint32_t par = (it / kPairStages) & 1;
-        if (!mbar_wait_cluster(smem_u32(&full_a[s]), par, abort_flag, args.status)) break;
-        if (!mbar_wait_cluster(smem_u32(&full_b[s]), par, abort_flag, args.status)) break;
+        const int ia = it % kPairRingA, iw = it % kPairRingW;
+        if (!mbar_wait(smem_u32(&full_a[ia]), par(it, kPairRingA), abort_flag, args.status)) break;
+        if (!mbar_wait(smem_u32(&full_w[iw]), par(it, kPairRingW), abort_flag, args.status)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(slot_a(s));
-        const uint32_t w_base = smem_u32(slot_w(s));
+        const uint32_t a_base = smem_u32(slot_a(it));
+        const uint32_t w_base = smem_u32(slot_w(it));
         const int nk = (it < args.num_kt) ? 4 : min(4, (args.lora_r16 - ((it - args.num_kt) % nl1) * 64) / 16);
         for (int k = 0; k < nk; ++k) {
           const uint64_t adesc = sw128_desc(a_base + k * 32, 16, 1024);
@@ -159,13 +196,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                                     : sw128_desc(w_base + k * 2048, 8192, 1024);
           umma_bf16_pair(tmem_d, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
         }
-        umma_commit_pair(smem_u32(&empty[s]), 0x3);
+        umma_commit_pair(smem_u32(&empty_a[ia]), 0x3);
+        umma_commit_pair(smem_u32(&empty_w[iw]), 0x3);
       }
       umma_commit_pair(smem_u32(acc_full), 0x3);
     }
   } else {
     // ---------------------------------------------------------- dequant
-    const int g = (warp - 2) >> 2;                 // stage parity this warp group handles
+    const int g = (warp - 2) >> 2;                 // handles stages it with it % kPairDeqGroups == g
     const int t = ((warp - 2) & 3) * 32 + lane;    // 0..127
     const int64_t KB = args.wK / 64;
     int64_t wn0, kb0, wn_step, kb_step;
@@ -180,7 +218,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       c_off = nl * 64; c_swz = (nl >> 1) & 3; c_ch0 = 2 * j;    // 64-byte rows, 64-byte swizzle
       w_off = j * 8192 + nl * 128; w_swz = nl & 7;
     }
-    // raw block-scale inputs of this thread's stage `it`, loaded 3 own stages ahead
+    // raw block-scale inputs of this thread's stages, loaded 3 own stages ahead
     auto load_raw = [&](int it, uint32_t& rq, float& rs) {
       rq = 0; rs = 0.0f;
       if (it >= args.num_kt) return;
@@ -192,22 +230,49 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     };
     uint32_t q0, q1, q2;
     float s0, s1, s2;
+    constexpr int G = kPairDeqGroups;
     load_raw(g, q0, s0);
-    load_raw(g + 2, q1, s1);
-    load_raw(g + 4, q2, s2);
-    for (int it = g; it < total; it += 2) {
-      const int s = it % kPairStages;
+    load_raw(g + G, q1, s1);
+    load_raw(g + 2 * G, q2, s2);
+    for (int it = g; it < total; it += G) {
+      const int ic = it % kPairRingC, iw = it % kPairRingW;
       const float scale = args.dq ? __fmul_rn(static_cast<float>(q0), s0) : s0;
-      q0 = q1; s0 = s1; q1 = q2; s1 = s2;
-      load_raw(it + 6, q2, s2);
-      if (!mbar_wait(smem_u32(&full_c[s]), (it / kPairStages) & 1, abort_flag, args.status)) break;
-      if (it < args.num_kt) {
-        const int64_t n = wn0 + wn_step * it, k = kb0 + kb_step * it;
-        uint8_t* wdst = slot_w(s) + w_off;
-        if (n < args.wN && k < KB) {
-          const uint8_t* cs = slot_c(s) + c_off;
-          const uint4 c0 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 0) ^ c_swz) << 4));
-          const uint4 c1 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 1) ^ c_swz) << 4));
+      if (!mbar_wait(smem_u32(&full_c[ic]), par(it, kPairRingC), abort_flag, args.status)) break;
+      const int64_t n = wn0 + wn_step * it, k = kb0 + kb_step * it;
+      const bool valid = it < args.num_kt && n < args.wN && k < KB;
+      uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
+      if (valid) {
+        const uint8_t* cs = slot_c(it) + c_off;
+        c0 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 0) ^ c_swz) << 4));
+        c1 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 1) ^ c_swz) << 4));
+      }
+      // Release the codes slot only once the loads above have returned: an
+      // arrive does not wait for loads whose results are still unused, and
+      // the next TMA would overwrite the slot under them.  Storing a value
+      // computed from every loaded word makes the release wait for them.
+      dep_scratch[(warp - 2) * 32 + lane] = c0.x ^ c0.y ^ c0.z ^ c0.w ^ c1.x ^ c1.y ^ c1.z ^ c1.w;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty_c[ic]));   // codes are in registers: slot may refill
+      // the bf16 slot is free once the MMA of its previous use has completed
+      if (it >= kPairRingW &&
+          !mbar_wait(smem_u32(&empty_w[iw]), prev_par(it, kPairRingW), abort_flag, args.status))
+        break;
+      if (it >= args.num_kt) {
+        // adapter stage: this CTA's adapter B half into the (now free) weight
+        // slot; its bytes complete on the leader's full_a of the same stage
+        if (((warp - 2) & 3) == 0 && lane == 0) {
+          const int li = (it - args.num_kt) % nl1;
+          const uint32_t fa = leader_bar(&full_a[it % kPairRingA]);
+          if (MODE == kModeFwd) {
+            tma_load_2d_pair(smem_u32(slot_w(it)), &tm_lb, fa, li * 64, static_cast<int32_t>(nc0));
+          } else {
+            tma_load_2d_pair(smem_u32(slot_w(it)), &tm_lb, fa, static_cast<int32_t>(nc0), li * 64);
+            tma_load_2d_pair(smem_u32(slot_w(it)) + 8192, &tm_lb, fa, static_cast<int32_t>(nc0) + 64, li * 64);
+          }
+        }
+      } else {
+        uint8_t* wdst = slot_w(it) + w_off;
+        if (valid) {
           const NF4Table tab = nf4_table(scale);
           const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
@@ -224,7 +289,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         fence_proxy_async_smem();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_bar(&full_b[s]));
+      if (lane == 0) mbar_arrive_cluster(leader_bar(&full_w[iw]));
+      // prefetch after the arrive, so that the arrive's release does not wait on these loads
+      q0 = q1; s0 = s1; q1 = q2; s1 = s2;
+      load_raw(it + 3 * G, q2, s2);
     }
 
     // ------------------------------------------------------------ epilogue
@@ -243,12 +311,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     tc_fence_after();
     if (!*abort_flag) {
       const int q = warp & 3;
-      const int half = (warp - 2) >> 2;
       const int64_t row = m0 + q * 32 + lane;
       const uint32_t taddr = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        const int col = half * 128 + c * 16;
+      for (int c = g; c < 16; c += kPairDeqGroups) {
+        const int col = c * 16;
         uint32_t r[16];
         tmem_ld16(taddr + col, r);
         tmem_ld_wait();
