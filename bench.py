@@ -422,16 +422,26 @@ def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_param
             X = inputs.normal((M, K), 1.0, 99 + M, dev)
             Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             ws = torch.empty(q.qlora_workspace_bytes(M, N, K, wl.r), dtype=torch.uint8, device=dev)
-            fn = lambda: q.qlora_linear_fwd(X, Wq, A, B, wl.alpha, Y=Y, workspace=ws)
+            kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(10)]
+            it = iter(kev * 2)
+            fn = lambda: q.qlora_linear_fwd(X, Wq, A, B, wl.alpha, Y=Y, workspace=ws, gemm_events=next(it))
             for _ in range(3):
                 fn()
+            it = iter(kev)
             ms = statistics.median(time_events(fn, 10, flush=lambda: l2buf.add_(1)))
+            kms = statistics.median(a.elapsed_time(b) for a, b in kev)
             wbytes = Wq.nbytes()
             res.append({"matrix": [N, K], "us": round(ms * 1e3, 2),
-                        "weight_gbs": round(wbytes / (ms * 1e-3) / 1e9, 1)})
+                        "weight_gbs": round(wbytes / (ms * 1e-3) / 1e9, 1),
+                        "kernel_us": round(kms * 1e3, 2),
+                        "kernel_weight_gbs": round(wbytes / (kms * 1e-3) / 1e9, 1)})
         gbs = [r_["weight_gbs"] for r_ in res]
+        kgbs = [r_["kernel_weight_gbs"] for r_ in res]
         dec[f"M{M}"] = {"per_matrix": res, "weight_gbs": round(sum(gbs) / len(gbs), 1),
-                        "frac_of_hbm": round(sum(gbs) / len(gbs) / hbm, 4)}
+                        "frac_of_hbm": round(sum(gbs) / len(gbs) / hbm, 4),
+                        "kernel_weight_gbs": round(sum(kgbs) / len(kgbs), 1),
+                        "kernel_frac_of_hbm": round(sum(kgbs) / len(kgbs) / hbm, 4)}
     out["decode_gemv"] = {"unit": "GB/s of NF4 weight (121.17 MB per matrix)", **dec,
                           "peak_hbm_gbs": hbm}
     return out

@@ -45,12 +45,14 @@ __device__ __forceinline__ NF4Table nf4_table(float scale) {
 __device__ __forceinline__ void nf4_decode8(uint32_t w, const NF4Table& t, uint32_t (&o)[4]) {
   const uint32_t idx = w & 0x77777777u;                              // low 3 bits of every code
   const uint32_t half = ((w >> 1) & 0x44444444u) | 0x32103210u;      // byte i from word A or B
+  // prmt reads only the low 16 bits (four nibbles) of its selector, so the
+  // upper half of idx / half needs no masking for h = 0
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint32_t s = (h ? (idx >> 16) : idx) & 0xFFFFu;
+    const uint32_t s = h ? (idx >> 16) : idx;
     const uint32_t g = h ? (half >> 16) : half;
-    const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], s), prmt(t.lo[2], t.lo[3], s), g & 0xFFFFu);
-    const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], s), prmt(t.hi[2], t.hi[3], s), g & 0xFFFFu);
+    const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], s), prmt(t.lo[2], t.lo[3], s), g);
+    const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], s), prmt(t.hi[2], t.hi[3], s), g);
     o[2 * h] = prmt(lo, hi, 0x5140u);
     o[2 * h + 1] = prmt(lo, hi, 0x7362u);
   }

@@ -24,6 +24,7 @@
 #include "gemm_nf4.cuh"
 #include "skinny.cuh"
 #include "gemm_nf4_pair.cuh"
+#include "gemv_nf4.cuh"
 
 using namespace qlora;
 
@@ -88,8 +89,22 @@ bool ensure_smem_attrs() {
   ok = ok && cudaFuncSetAttribute(k_skinny<0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_gemv_nf4, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes) == cudaSuccess;
   if (ok) done.fetch_or(bit);
   return ok;
+}
+
+// streaming multiprocessors of the current device (cached per device)
+int sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int v = cache[dev].load();
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev].store(v);
+  }
+  return v;
 }
 
 qlora_status check_launch() {
@@ -168,8 +183,11 @@ qlora_status launch_skinny(const SkPlan& pl, const CUtensorMap& ta, const CUtens
 
 // -------------------------------------------------------- workspace layout
 struct Ws {
-  size_t partial, t32, sx, ghl, thl, bpad, total;
+  size_t partial, t32, sx, ghl, thl, bpad, gv_part, gv_cnt, total;
 };
+
+// Token counts up to this take the weight-streaming decode kernel.
+constexpr int64_t kDecodeMaxM = kGvNT;
 
 struct Dims {
   int64_t M, N, K;
@@ -201,6 +219,11 @@ Ws ws_layout(const Dims& d) {
   w.ghl = off; off += a256(static_cast<size_t>(d.M) * d.Qh * 2);
   w.thl = off; off += a256(static_cast<size_t>(d.M) * d.Qh * 2);
   w.bpad = off; off += a256(static_cast<size_t>(d.N) * d.r8 * 2);
+  w.gv_part = w.gv_cnt = off;
+  if (d.M <= kDecodeMaxM) {
+    w.gv_part = off; off += a256(static_cast<size_t>(kGvMaxCtas) * 2 * kGvRows * kGvNT * 4);
+    w.gv_cnt = off; off += a256(static_cast<size_t>(cdiv(d.N, kGvRows)) * 4);
+  }
   w.total = off;
   return w;
 }
@@ -336,6 +359,45 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   return QLORA_OK;
 }
 
+// Decode-shaped forward (M <= 16): Y = X W^T + s T B^T with T = X A^T in
+// fp32 at t32.  Persistent stream-K launch, one CTA per SM.
+qlora_status run_gemv(const void* X, const qlora_nf4_weight* Wq, const Dims& d, const float* t32, const void* B,
+                      void* Y, float alpha_over_r, uint8_t* ws, const Ws& L, const qlora_gemm_events* ev,
+                      int* status, cudaStream_t cs) {
+  if (d.r > kGvMaxRank) return QLORA_ERR_UNSUPPORTED;
+  const int64_t tiles = cdiv(d.N, kGvRows);
+  const int64_t KU = cdiv(d.K, kGvKS);
+  const int64_t units = tiles * KU;
+  const int sms = sm_count();
+  if (sms <= 0) return QLORA_ERR_CUDA;
+  const int64_t grid = std::min<int64_t>(std::min<int64_t>(sms, kGvMaxCtas), units);
+  CUtensorMap tx, tc;
+  if (!bf16_map(&tx, X, d.K, d.M, d.K, 64, kGvNT)) return QLORA_ERR_CUDA;
+  if (!make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, kGvKS / 2, kGvRows,
+                CU_TENSOR_MAP_SWIZZLE_64B))
+    return QLORA_ERR_CUDA;
+  GvArgs a{};
+  a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
+  a.N = d.N; a.K = d.K; a.M = static_cast<int>(d.M); a.r = d.r; a.s = alpha_over_r;
+  a.T = t32;
+  a.B = static_cast<const __nv_bfloat16*>(B);
+  a.Y = static_cast<__nv_bfloat16*>(Y);
+  a.part = reinterpret_cast<float*>(ws + L.gv_part);
+  a.cnt = reinterpret_cast<int*>(ws + L.gv_cnt);
+  a.KU = KU;
+  a.units = units;
+  a.status = status;
+  if (cudaMemsetAsync(a.cnt, 0, static_cast<size_t>(tiles) * 4, cs) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (ev && ev->gemm_start && cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_start), cs) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  k_gemv_nf4<<<static_cast<unsigned>(grid), kGvThreads, kGvSmemBytes, cs>>>(tx, tc, a);
+  qlora_status rc = check_launch();
+  if (rc == QLORA_OK && ev && ev->gemm_end &&
+      cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_end), cs) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return rc;
+}
+
 }  // namespace
 
 // =================================================================== ABI
@@ -428,6 +490,13 @@ qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* 
   const float s = alpha / static_cast<float>(r);
   float* t32 = T_save ? T_save : reinterpret_cast<float*>(ws + L.t32);
   __nv_bfloat16* sT = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
+
+  if (M <= kDecodeMaxM) {
+    // decode shape: T = X A^T (fp32), then the weight-streaming kernel
+    st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
+    if (st != QLORA_OK) return st;
+    return run_gemv(X, Wq, d, t32, B, Y, s, ws, L, events, d_status, cs);
+  }
 
   // 1. T = X A^T and s*T (bf16) for the fold
   st = run_T(X, A, d, s, ws, L, t32, sT, d_status, cs);
@@ -559,6 +628,11 @@ Ws noalloc_fwd_layout(const Dims& d) {
   w.sx = off; off += a256(static_cast<size_t>(2 * d.M) * d.r8 * 2);
   w.ghl = w.thl = off;
   w.bpad = off; off += (d.r % 8) ? a256(static_cast<size_t>(d.N) * d.r8 * 2) : 0;
+  w.gv_part = w.gv_cnt = off;
+  if (d.M <= kDecodeMaxM) {
+    w.gv_part = off; off += a256(static_cast<size_t>(kGvMaxCtas) * 2 * kGvRows * kGvNT * 4);
+    w.gv_cnt = off; off += a256(static_cast<size_t>(cdiv(d.N, kGvRows)) * 4);
+  }
   w.total = off;
   return w;
 }
@@ -587,6 +661,12 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const void* X, int64_t M, const
   const float s = alpha / static_cast<float>(r);
   float* t32 = T_save ? T_save : reinterpret_cast<float*>(ws + L.t32);
   __nv_bfloat16* sT = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
+
+  if (M <= kDecodeMaxM) {
+    st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
+    if (st != QLORA_OK) return st;
+    return run_gemv(X, Wq, d, t32, B, Y, s, ws, L, nullptr, d_status, cs);
+  }
 
   st = run_T(X, A, d, s, ws, L, t32, sT, d_status, cs);
   if (st != QLORA_OK) return st;

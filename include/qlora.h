@@ -151,9 +151,14 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  *     T = X A^T  [M, r]          Y = X W^T + s T B^T  [M, N]
  * X bf16 [M, K]; A bf16 [r, K]; B bf16 [N, r]; Y bf16 [M, N] (written).
  * T_save (nullable) fp32 [M, r]: T for the backward.  1 <= r <= 256.
- * W^ is dequantised tile by tile in shared memory inside the GEMM; the
- * adapter product enters the same fp32 accumulator, one bf16 rounding per
- * output.  Requires N % 8 == 0, K % 64 == 0.
+ * M > 16: W^ is dequantised tile by tile in shared memory inside the
+ * GEMM; the adapter product enters the same fp32 accumulator, one bf16
+ * rounding per output.  M <= 16 (decode): a weight-streaming kernel
+ * dequantises W^ straight into tensor memory, accumulates X W^T in fp32,
+ * adds s T B^T in fp32 and rounds once; the workspace then also holds
+ * per-CTA partial tiles and per-tile counters, which the call clears on
+ * the stream before use.  Results are deterministic (fixed summation
+ * order) for both paths.  Requires N % 8 == 0, K % 64 == 0.
  */
 qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* Wq,
                               const void* A, const void* B, int r, float alpha,
@@ -195,8 +200,9 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M,
  * whose forward scratch (split-K partials of T, fp32 T, the two bf16 planes
  * of s*T, a padded copy of B when r % 8 != 0) does not fit is rejected with
  * QLORA_ERR_SCRATCH_LIMIT before anything is enqueued; e.g. M = 8192,
- * r = 64 fits.  Every region is fully written before it is read, so nothing
- * needs clearing between calls.
+ * r = 64 fits.  Every region is fully written before it is read, except
+ * the decode path's (M <= 16) tile counters, which each call clears on
+ * its stream before its kernels run.
  *
  * All calls on a device share the one array: calls whose work overlaps on
  * the GPU (different streams, or different host threads) race and give
