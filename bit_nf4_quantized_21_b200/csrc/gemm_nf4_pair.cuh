@@ -37,10 +37,15 @@
 namespace qlora {
 
 constexpr int kPairRingA = 5;                    // activation ring depth
-constexpr int kPairRingC = 8;                    // packed-code ring depth
+constexpr int kPairRingC = 9;                    // packed-code ring depth
 constexpr int kPairRingW = 6;                    // dequantised-weight ring depth
 constexpr int kPairDeqGroups = 3;                // group it % 3 decodes stage it (owns W slots g, g + 3)
+// A waiter that takes every G-th stage must own whole slots: with a ring
+// depth that is not a multiple of G it could come to a slot whose previous
+// phase (another waiter's stage) is still pending, and a parity wait would
+// then take the phase before that for the one it wants.
 static_assert(kPairRingW % kPairDeqGroups == 0, "each weight slot must belong to one dequant group");
+static_assert(kPairRingC % kPairDeqGroups == 0, "each code slot must belong to one dequant group");
 constexpr int kPairDeqWarps = 4;                 // warps per group (128 weight rows)
 constexpr int kPairThreads = 64 + kPairDeqGroups * kPairDeqWarps * 32;
 constexpr uint32_t kPairABytes = 128 * 64 * 2;   // 16 KB activations (this CTA's half)
@@ -132,13 +137,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tma_load_2d_pair(smem_u32(slot_a(it)), &tm_act, fa, it * 64, static_cast<int32_t>(m0));
         } else {
           // adapter stage: the A tile here; the adapter B tile is loaded into
-          // the weight slot by the dequant group that owns the slot (it waits
-          // for every phase of that slot in order; this thread runs up to a
-          // whole activation ring ahead and would alias the slot's phases)
+          // the weight slot, and its bytes counted on that slot's full_w, by
+          // the dequant group that owns the slot (it has seen every earlier
+          // phase of full_w; this thread may be a whole activation ring
+          // ahead, and full_a of this slot may still be in an earlier stage's
+          // phase, so neither may carry the B tile's bytes)
           const int lt = it - args.num_kt;
           const int li = lt % nl1;
           const int64_t arow = (lt / nl1) * args.lora_lo_row + m0;
-          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * (kPairABytes + kPairWBytes));
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * kPairABytes);
           tma_load_2d_pair(smem_u32(slot_a(it)), &tm_la, fa, li * 64, static_cast<int32_t>(arow));
         }
         ++issued;
@@ -259,15 +266,19 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         break;
       if (it >= args.num_kt) {
         // adapter stage: this CTA's adapter B half into the (now free) weight
-        // slot; its bytes complete on the leader's full_a of the same stage
+        // slot; its bytes complete on the leader's full_w of this stage,
+        // which this group has already seen advance past the slot's
+        // previous use (the empty_w wait above).  The expect comes before
+        // this warp's own arrive, so the phase cannot complete without it.
         if (((warp - 2) & 3) == 0 && lane == 0) {
           const int li = (it - args.num_kt) % nl1;
-          const uint32_t fa = leader_bar(&full_a[it % kPairRingA]);
+          const uint32_t fw = leader_bar(&full_w[iw]);
+          mbar_expect_tx_cluster(fw, kPairWBytes);
           if (MODE == kModeFwd) {
-            tma_load_2d_pair(smem_u32(slot_w(it)), &tm_lb, fa, li * 64, static_cast<int32_t>(nc0));
+            tma_load_2d_pair(smem_u32(slot_w(it)), &tm_lb, fw, li * 64, static_cast<int32_t>(nc0));
           } else {
-            tma_load_2d_pair(smem_u32(slot_w(it)), &tm_lb, fa, static_cast<int32_t>(nc0), li * 64);
-            tma_load_2d_pair(smem_u32(slot_w(it)) + 8192, &tm_lb, fa, static_cast<int32_t>(nc0) + 64, li * 64);
+            tma_load_2d_pair(smem_u32(slot_w(it)), &tm_lb, fw, static_cast<int32_t>(nc0), li * 64);
+            tma_load_2d_pair(smem_u32(slot_w(it)) + 8192, &tm_lb, fw, static_cast<int32_t>(nc0) + 64, li * 64);
           }
         }
       } else {
@@ -293,6 +304,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       // prefetch after the arrive, so that the arrive's release does not wait on these loads
       q0 = q1; s0 = s1; q1 = q2; s1 = s2;
       load_raw(it + 3 * G, q2, s2);
+    }
+    // After an abort, adapter-tile loads this lane issued may still be in
+    // flight into shared memory, and nobody else waits for them: give them
+    // time to land before the CTA can exit (error path only; a tile load
+    // takes microseconds).
+    if (*abort_flag && ((warp - 2) & 3) == 0 && lane == 0 && total > args.num_kt) {
+      const uint64_t t0 = global_ns();
+      while (global_ns() - t0 < 1000000ull) {}
     }
 
     // ------------------------------------------------------------ epilogue
@@ -337,6 +356,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
   }
 
+  // Single-lane roles (producer, MMA issuer) leave their warps diverged;
+  // the CTA/cluster barrier below is warp-aligned, so every warp first
+  // reconverges here -- otherwise the barrier can complete while a lane is
+  // still working and TMEM could be released under it.
+  __syncwarp();
   tc_fence_before();
   cluster_sync();   // the peer may still read this CTA's shared memory / arrive on its barriers until here
   if (warp == 1) {

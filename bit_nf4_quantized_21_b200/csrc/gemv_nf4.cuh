@@ -10,11 +10,12 @@
 // keep the weight stream moving and to spend as little as possible per
 // weight on the chip.
 //
-// Roles per CTA (576 threads, one CTA per SM, persistent):
+// Roles per CTA (608 threads, one CTA per SM, persistent):
 //   warp 0       TMA producer: per 128-deep slice, the packed codes of 128
 //                weight rows (8 KB, 64 bytes per row) and the matching
 //                16 x 128 activation slice (4 KB) into a shared-memory ring
-//   warp 1       TMEM allocator and single-thread MMA issuer
+//   warps 1, 18  MMA issuers (warp 1 also allocates TMEM): issuer i takes
+//                the slices with it = i (mod 2) into its own accumulator
 //   warps 2..13  three dequant groups of 4 warps; group g decodes slices
 //                it = g (mod 3).  Thread = one weight row: its 128 codes of
 //                the slice are exactly two quantisation blocks, each decoded
@@ -27,12 +28,14 @@
 //                to bf16.
 // MMA per slice: 8 x tcgen05.mma.cta_group::1.kind::f16, M 128 (weight
 // rows, A from TMEM), N 16 (tokens, B = activation slice, K-major, 128-byte
-// swizzle), K 16; the accumulator is double-buffered in TMEM so the
-// epilogue of one tile overlaps the next tile's stream.  The slice depth is
-// set by the MMA issue cost, not the math: one tcgen05.mma takes ~50 cycles
-// to issue at any N <= 64 and a commit ~46 (measured on B200), so a
-// 64-deep slice (4 MMAs + 2 commits per 8192 weights) capped the stream at
-// ~14 weights per clock per SM; 128-deep slices halve that overhead.
+// swizzle), K 16; each issuer's accumulator is double-buffered in TMEM so
+// the epilogue of one tile overlaps the next tile's stream.  At N = 16 the
+// limit is the issuing thread, not the math (measured on B200): a
+// tcgen05.mma occupies the tensor pipe ~45-50 cycles at any N <= 64, but
+// one thread that waits on a barrier, issues a slice's 8 MMAs and commits
+// needs ~720 cycles per slice; two issuers on different SMSPs need ~350
+// between them.  Hence 128-deep slices (fewer waits and commits per
+// weight) and two issuers.
 //
 // Work split (stream-K): the weight is cut into units of 128 rows x 128
 // columns, ordered tile-major (tile = 128 rows); CTA c of G streams units
@@ -50,12 +53,17 @@ namespace qlora {
 constexpr int kGvRows = 128;                  // weight rows per tile (MMA M)
 constexpr int kGvNT = 16;                     // token columns (MMA N); M <= 16
 constexpr int kGvKS = 128;                    // contraction depth of one slice (two 64-weight blocks)
-constexpr int kGvStages = 7;                  // ring depth: slot i = codes + activations (smem) + dequantised slice (TMEM)
-constexpr int kGvMmaBatch = 1;                // slices per MMA-thread wait (1 measured fastest: see the MMA issuer)
+constexpr int kGvStages = 6;                  // ring depth: slot i = codes + activations (smem) + dequantised slice (TMEM)
+constexpr int kGvIssuers = 2;                 // MMA-issuing threads (warps 1 and kGvIssuerWarp1)
 constexpr int kGvGroups = 3;                  // dequant warp groups
 constexpr int kGvDeqWarps = 4 * kGvGroups;
+// Waiters that take every G-th slice (dequant groups, issuers) must own
+// whole ring slots, or a parity wait could take an older phase for the
+// pending one.
+static_assert(kGvStages % kGvGroups == 0 && kGvStages % kGvIssuers == 0, "ring slots per waiter");
 constexpr int kGvEpiWarp0 = 2 + kGvDeqWarps;  // first epilogue warp
-constexpr int kGvThreads = 32 * (kGvEpiWarp0 + 4);
+constexpr int kGvIssuerWarp1 = kGvEpiWarp0 + 4;  // second MMA issuer (its own warp, another SMSP)
+constexpr int kGvThreads = 32 * (kGvIssuerWarp1 + 1);
 constexpr int kGvMaxCtas = 256;               // partial-tile slots in the workspace
 constexpr int kGvMaxRank = 256;
 constexpr uint32_t kGvCBytes = kGvRows * kGvKS / 2;  // 8 KB packed codes per slice
@@ -65,8 +73,8 @@ constexpr uint32_t kGvOffST = kGvOffX + kGvStages * kGvXBytes;
 constexpr uint32_t kGvOffBar = kGvOffST + kGvNT * kGvMaxRank * 4;
 constexpr uint32_t kGvSmemUsed = kGvOffBar + 1024 /*align*/ + 512 /*barriers*/;
 constexpr uint32_t kGvSmemBytes = kGvSmemUsed > 118 * 1024 ? kGvSmemUsed : 118 * 1024;   // one CTA per SM
-constexpr uint32_t kGvTmemCols = 512;         // D buffers at columns 0 and 32, A slots at 64 + 64 i
-constexpr uint32_t kGvTmemA0 = 64;
+constexpr uint32_t kGvTmemCols = 512;         // D[issuer][buffer] at columns 32 (2 issuer + buffer), A slots at 128 + 64 i
+constexpr uint32_t kGvTmemA0 = 32 * 2 * kGvIssuers;
 constexpr uint32_t kGvASlotCols = kGvKS / 2;  // 2 bf16 per 32-bit column
 static_assert(kGvTmemA0 + kGvASlotCols * kGvStages <= kGvTmemCols, "TMEM budget");
 static_assert(kGvSmemBytes <= 227 * 1024, "shared memory budget");
@@ -163,10 +171,11 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   uint64_t* fullc = bars;                              // [S] packed codes landed (TMA)
   uint64_t* ready = fullc + kGvStages;                 // [S] activations landed (TMA) + slice in TMEM (4 warps)
   uint64_t* empty = ready + kGvStages;                 // [S] codes read (4 warps) + MMA done with the slot (commit)
-  uint64_t* d_full = empty + kGvStages;                // [2] accumulator complete
-  uint64_t* d_empty = d_full + 2;                      // [2] accumulator read out (4 warps)
-  uint64_t* mma_done = d_empty + 2;                    // every MMA of this CTA retired
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* d_full = empty + kGvStages;                // [issuer][2] accumulator complete
+  uint64_t* d_empty = d_full + 2 * kGvIssuers;         // [issuer][2] accumulator read out (4 warps)
+  uint64_t* mma_done = d_empty + 2 * kGvIssuers;       // every MMA of this CTA retired (one commit per issuer)
+  uint64_t* epi_done = mma_done + 1;                   // every epilogue TMEM read retired (4 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* s_last = abort_flag + 1;
 
@@ -184,11 +193,12 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       mbar_init(smem_u32(&ready[i]), 1 + 4);
       mbar_init(smem_u32(&empty[i]), 4 + 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 2 * kGvIssuers; ++i) {
       mbar_init(smem_u32(&d_full[i]), 1);
       mbar_init(smem_u32(&d_empty[i]), 4);
     }
-    mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(mma_done), kGvIssuers);
+    mbar_init(smem_u32(epi_done), 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -218,7 +228,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       for (int it = 0; it < n_it; ++it) {
         const int s = it % kGvStages;
         if (it >= kGvStages &&
-            !mbar_wait(smem_u32(&empty[s]), ((it / kGvStages) + 1) & 1, abort_flag, args.status))
+            !mbar_wait_sleep(smem_u32(&empty[s]), ((it / kGvStages) + 1) & 1, abort_flag, args.status, 64))
           break;
         const uint32_t fc = smem_u32(&fullc[s]), rb = smem_u32(&ready[s]);
         mbar_arrive_expect_tx(fc, kGvCBytes);
@@ -245,57 +255,51 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    // In isolation the first barrier wait after a run of MMAs costs this
-    // thread ~250 cycles and a second one right after ~45, which suggests
-    // waiting for several slices before issuing their MMAs; in the full
-    // kernel batches of 2-4 measured slower than 1 (the MMAs start later and
-    // the ring drains), so kGvMmaBatch stays 1.  Descriptors are precomputed: per MMA the
-    // thread adds an offset to the activation descriptor's address field
-    // (bits 0..13, address >> 4; every slot lies below 256 KB, so the add
-    // never carries out of the field) and to the TMEM column.
+  } else if (warp == 1 || warp == kGvIssuerWarp1) {
+    // ---------------------------------------------------------- MMA issuers
+    // Issuer i takes the CTA's slices it = i (mod 2) and accumulates them
+    // into D[i][segment parity]; for every tile piece (segment) it commits
+    // d_full[i][.] once -- also when it had no slice in that piece, which
+    // the epilogue knows from the same slice numbering.  Per slice: one
+    // barrier wait, 8 MMAs, one commit.  The activation descriptor's address
+    // field (bits 0..13, address >> 4) is advanced by plain adds: every slot
+    // lies below 256 KB, so the add never carries out of the field.
     if (lane == 0) {
+      const int me = (warp == 1) ? 0 : 1;
       constexpr uint32_t idesc = idesc_bf16(kGvRows, kGvNT, 0, 0);
       const uint64_t xdesc0 = sw128_desc(smem_u32(base + kGvOffX), 16, 1024);
-      int64_t ku = u0 % KU;
-      int j = -1;   // segment (tile piece) index of this CTA
+      int64_t u = u0;
+      int j = 0;
       bool ok = true;
-      for (int it0 = 0; it0 < n_it && ok; it0 += kGvMmaBatch) {
-        const int nb = min(kGvMmaBatch, n_it - it0);
-        for (int b = 0; b < nb; ++b) {
-          const int it = it0 + b;
-          if (!mbar_wait(smem_u32(&ready[it % kGvStages]), (it / kGvStages) & 1, abort_flag, args.status)) {
+      while (u < u1 && ok) {
+        const int64_t t = u / KU;
+        const int64_t seg_end = min(u1, (t + 1) * KU);
+        const int it_a = static_cast<int>(u - u0), it_b = static_cast<int>(seg_end - u0);
+        const uint32_t d_col = tmem + 32u * (2 * me + (j & 1));
+        if (j >= 2 && !mbar_wait(smem_u32(&d_empty[2 * me + (j & 1)]), ((j >> 1) + 1) & 1, abort_flag, args.status))
+          break;
+        bool first = true;
+        for (int it = it_a + (((it_a & 1) != me) ? 1 : 0); it < it_b; it += kGvIssuers) {
+          const int s = it % kGvStages;
+          if (!mbar_wait(smem_u32(&ready[s]), (it / kGvStages) & 1, abort_flag, args.status)) {
             ok = false;
             break;
           }
-        }
-        if (!ok) break;
-        tc_fence_after();
-        for (int b = 0; b < nb; ++b) {
-          const int it = it0 + b;
-          const bool seg_first = (it == 0) || (ku == 0);
-          const bool seg_last = (it == n_it - 1) || (ku == KU - 1);
-          if (seg_first) {
-            ++j;
-            if (j >= 2 && !mbar_wait(smem_u32(&d_empty[j & 1]), ((j >> 1) + 1) & 1, abort_flag, args.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          const int s = it % kGvStages;
+          tc_fence_after();
           const uint64_t xdesc = xdesc0 + static_cast<uint64_t>((s * kGvXBytes) >> 4);
           const uint32_t a_col = tmem + kGvTmemA0 + kGvASlotCols * s;
-          const uint32_t d_col = tmem + 32u * (j & 1);
 #pragma unroll
           for (int k = 0; k < kGvKS / 16; ++k)
-            umma_bf16_ts(d_col, a_col + 8u * k, xdesc + static_cast<uint64_t>(((k >> 2) * (kGvXBytes / 2) + 32 * (k & 3)) >> 4),
-                         idesc, (seg_first && k == 0) ? 0u : 1u);
+            umma_bf16_ts(d_col, a_col + 8u * k,
+                         xdesc + static_cast<uint64_t>(((k >> 2) * (kGvXBytes / 2) + 32 * (k & 3)) >> 4), idesc,
+                         (first && k == 0) ? 0u : 1u);
           umma_commit(smem_u32(&empty[s]));
-          if (seg_last) umma_commit(smem_u32(&d_full[j & 1]));
-          if (++ku == KU) ku = 0;
+          first = false;
         }
+        if (!ok) break;
+        umma_commit(smem_u32(&d_full[2 * me + (j & 1)]));
+        u = seg_end;
+        ++j;
       }
       umma_commit(smem_u32(mma_done));
     }
@@ -391,21 +395,55 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       const int64_t t = u / KU;
       const int64_t seg_end = min(u1, (t + 1) * KU);
       const bool whole = (u == t * KU) && (seg_end == (t + 1) * KU);
+      const int64_t n = t * kGvRows + row;
+      // adapter term z[m] = sum_j (s T)[m, j] B[n, j] in fp32, computed while
+      // the tile is still streaming (it does not depend on the accumulator)
+      float z[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) z[m] = 0.0f;
+      if (n < args.N) {
+        const __nv_bfloat16* brow = args.B + n * args.r;
+        for (int j0 = 0; j0 < args.r; j0 += 8) {
+          float bv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) bv[i] = (j0 + i < args.r) ? __bfloat162float(brow[j0 + i]) : 0.0f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (j0 + i < args.r) {
+#pragma unroll
+              for (int m = 0; m < 16; ++m)
+                if (m < args.M) z[m] = fmaf(sT[m * args.r + j0 + i], bv[i], z[m]);
+            }
+          }
+        }
+      }
       // every epilogue thread reaches this barrier, and all leave the loop
       // together if any of them gave up waiting
-      const bool got = mbar_wait(smem_u32(&d_full[j & 1]), (j >> 1) & 1, abort_flag, args.status);
+      bool got = mbar_wait_sleep(smem_u32(&d_full[0 + (j & 1)]), (j >> 1) & 1, abort_flag, args.status, 256);
+      got = got && mbar_wait_sleep(smem_u32(&d_full[2 + (j & 1)]), (j >> 1) & 1, abort_flag, args.status, 256);
       if (!named_bar_and(1, 128, got)) break;
       tc_fence_after();
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_base + 32u * (j & 1), v);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&d_empty[j & 1]));
-      const int64_t n = t * kGvRows + row;
+      // issuer i holds part of this piece iff it had a slice in it
+      const int it_a = static_cast<int>(u - u0), it_b = static_cast<int>(seg_end - u0);
       float y[16];
 #pragma unroll
-      for (int m = 0; m < 16; ++m) y[m] = __uint_as_float(v[m]);
+      for (int m = 0; m < 16; ++m) y[m] = 0.0f;
+#pragma unroll
+      for (int i = 0; i < kGvIssuers; ++i) {
+        if (it_b - it_a >= 2 || (it_a & 1) == i) {
+          uint32_t v[16];
+          tmem_ld16(tmem + lane_base + 32u * (2 * i + (j & 1)), v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int m = 0; m < 16; ++m) y[m] += __uint_as_float(v[m]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&d_empty[0 + (j & 1)]));
+        mbar_arrive(smem_u32(&d_empty[2 + (j & 1)]));
+      }
       bool finish = whole;
       if (!whole) {
         // partial tile: publish, count, and the last arrival adds them up
@@ -440,35 +478,43 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         }
       }
       if (finish && n < args.N) {
-        // adapter term in fp32, then one rounding to bf16
-        const __nv_bfloat16* brow = args.B + n * args.r;
-        for (int jr = 0; jr < args.r; ++jr) {
-          const float bv = __bfloat162float(brow[jr]);
-#pragma unroll
-          for (int m = 0; m < 16; ++m)
-            if (m < args.M) y[m] = fmaf(sT[m * args.r + jr], bv, y[m]);
-        }
+        // frozen-base sum plus adapter term, one rounding to bf16
 #pragma unroll
         for (int m = 0; m < 16; ++m)
-          if (m < args.M) args.Y[static_cast<int64_t>(m) * args.N + n] = __float2bfloat16_rn(y[m]);
+          if (m < args.M) args.Y[static_cast<int64_t>(m) * args.N + n] = __float2bfloat16_rn(y[m] + z[m]);
       }
       u = seg_end;
       ++j;
     }
+    // this warp's TMEM reads are complete (tcgen05.wait::ld above)
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(epi_done));
   }
 
-  // every MMA must have retired before TMEM is released
-  if (warp == 1) {
-    const uint32_t bar = smem_u32(mma_done);
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar, 0)) {
-      if (global_ns() - t0 > QLORA_WAIT_NS) {
-        *abort_flag = 1;
-        if (args.status) atomicOr(args.status, QLORA_DEV_TIMEOUT);
-        break;
+  // every MMA (both issuers) and every epilogue TMEM read must have retired
+  // before TMEM is released; the owner's lane 0 waits for both explicitly
+  // (bounded, ignoring abort) once its own issuing is over -- the other 31
+  // lanes wait at the __syncwarp below instead of polling all kernel long
+  if (warp == 1 && lane == 0) {
+    const uint32_t bars2[2] = {smem_u32(mma_done), smem_u32(epi_done)};
+    for (int i = 0; i < 2; ++i) {
+      const uint64_t t0 = global_ns();
+      while (!mbar_try_wait(bars2[i], 0)) {
+        __nanosleep(64);
+        if (global_ns() - t0 > QLORA_WAIT_NS) {
+          *abort_flag = 1;
+          if (args.status) atomicOr(args.status, QLORA_DEV_TIMEOUT);
+          break;
+        }
       }
     }
   }
+  // Single-lane roles (producer, MMA issuer) leave their warps diverged;
+  // the CTA/cluster barrier below is warp-aligned, so every warp first
+  // reconverges here -- otherwise the barrier can complete while a lane is
+  // still working and TMEM could be released under it.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -170,6 +170,11 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     }
   }
 
+  // Single-lane roles (producer, MMA issuer) leave their warps diverged;
+  // the CTA/cluster barrier below is warp-aligned, so every warp first
+  // reconverges here -- otherwise the barrier can complete while a lane is
+  // still working and TMEM could be released under it.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
