@@ -538,10 +538,39 @@ def run_reference(args):
 
 def run_only(args):
     """One projection's forward or backward call, repeated: the small case
-    for kernel profiles (ncu) of the fused GEMM."""
+    for kernel profiles (ncu) of the fused GEMM; with --only decode, the
+    decode-shaped forward of one 70B MLP matrix (--proj 0: 28672 x 8192,
+    1: 8192 x 28672) at --tokens <= 16."""
     import bit_nf4_quantized_21_b200 as q
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    if args.only == "decode":
+        wl = inputs.DECODE
+        name, N, K = wl.shapes[args.proj]
+        M = args.tokens
+        seed = inputs.matrix_seed(wl.base_seed, 0, args.proj)
+        W = inputs.weight((N, K), wl.w_std, seed, device=dev, outlier_frac=wl.outlier_frac,
+                          outlier_scale=wl.outlier_scale)
+        Wq = q.qlora_quantize_nf4(W)
+        del W
+        X = inputs.normal((M, K), 1.0, 99 + M, dev)
+        A = inputs.normal((wl.r, K), 0.01, seed * 16 + 3, dev)
+        B = inputs.normal((N, wl.r), 0.01, seed * 16 + 4, dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(q.qlora_workspace_bytes(M, N, K, wl.r), dtype=torch.uint8, device=dev)
+        l2 = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+        evs = []
+        for i in range(args.warmup + args.steps):
+            l2.add_(1)
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            q.qlora_linear_fwd(X, Wq, A, B, wl.alpha, Y=Y, workspace=ws, gemm_events=ev)
+            if i >= args.warmup:
+                evs.append(ev)
+        torch.cuda.synchronize()
+        us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+        print(json.dumps({"only": "decode", "shape": [M, N, K], "kernel_us": round(us, 2),
+                          "weight_gbs": round(Wq.nbytes() / (us * 1e-6) / 1e9, 1)}))
+        return
     name, N, K = WL.shapes[args.proj]
     M = args.tokens
     seed = inputs.matrix_seed(WL.base_seed, 0, args.proj)
@@ -580,7 +609,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--only", choices=("gemm-fwd", "gemm-dx"), default=None,
+    ap.add_argument("--only", choices=("gemm-fwd", "gemm-dx", "decode"), default=None,
                     help="profile mode: repeat one projection's call (see --proj, --tokens)")
     ap.add_argument("--proj", type=int, default=4)
     ap.add_argument("--tokens", type=int, default=2048)

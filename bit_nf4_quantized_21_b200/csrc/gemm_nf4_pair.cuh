@@ -11,24 +11,29 @@
 //
 // Three shared-memory rings per CTA; stage `it` (64 deep) uses slot
 // it % depth of each:
-//   activations  5 x 16 KB  pair TMA by producer lane 0, completing on the
+//   activations  4 x 16 KB  pair TMA by producer lane 0, completing on the
 //                           leader's full_a; freed by the MMA (empty_a)
-//   codes        8 x  4 KB  local TMA by producer lane 1 (full_c); freed by
+//   codes        9 x  4 KB  local TMA by producer lane 1 (full_c); freed by
 //                           the dequant warps once the codes are in
 //                           registers (empty_c)
 //   bf16 weight  6 x 16 KB  written by dequant group it % 3 after the MMA
 //                           freed the slot (empty_w); one arrive per warp
 //                           on the leader's full_w
-// Ring depths follow measured hand-off latencies: every hop (commit ->
-// barrier -> wake -> load or decode -> arrive -> wake) costs hundreds of
-// cycles, and the decode loop has the most hops, so the weight ring is the
-// deepest of the 16 KB rings.  The leader's
-// MMA thread waits full_a and full_w, issues 4 tcgen05.mma.cta_group::2
-// (M 256, N 256, K 16) and commits to empty_a and empty_w in both CTAs
-// (multicast commits).  Adapter stages load their B operand by TMA into the
-// weight slot, issued by the dequant group that owns the slot.
-// Every waiter waits for each phase of a barrier in order (no waiter can be
-// two phases behind), which is what makes the 1-bit phase parity safe.
+// Two MMA-issuing threads in the leader (warps 1 and 14) take alternate
+// stages: issuer i waits full_a and full_w of stage it = i (mod 2), issues
+// its 4 tcgen05.mma.cta_group::2 (M 256, N 256, K 16) into its own
+// accumulator D_i (TMEM columns 256 i .. 256 i + 255: the two use all 512)
+// and commits to empty_a and empty_w in both CTAs (multicast commits).  A
+// thread that waits on a barrier right after issuing MMAs stalls until they
+// drain (~250 cycles of bubble per stage, measured), which one issuer
+// cannot hide; with two, one issues while the other waits.  The epilogue
+// adds D_0 + D_1 (fixed order: deterministic).  Adapter stages load their
+// B operand by TMA into the weight slot, issued by the dequant group that
+// owns the slot, with the bytes counted on that slot's full_w.
+// Every waiter waits for each phase of its slots in order: a waiter that
+// takes every G-th stage (issuers G = 2, dequant groups G = 3) owns whole
+// slots because each ring depth is a multiple of its waiters' G, so no
+// waiter can be two phases behind and the 1-bit phase parity is safe.
 // Epilogue: every CTA reads its own TMEM half (tcgen05.ld) and writes bf16.
 #pragma once
 #include "nf4_decode.cuh"
@@ -36,7 +41,7 @@
 
 namespace qlora {
 
-constexpr int kPairRingA = 5;                    // activation ring depth
+constexpr int kPairRingA = 4;                    // activation ring depth
 constexpr int kPairRingC = 9;                    // packed-code ring depth
 constexpr int kPairRingW = 6;                    // dequantised-weight ring depth
 constexpr int kPairDeqGroups = 3;                // group it % 3 decodes stage it (owns W slots g, g + 3)
@@ -47,7 +52,10 @@ constexpr int kPairDeqGroups = 3;                // group it % 3 decodes stage i
 static_assert(kPairRingW % kPairDeqGroups == 0, "each weight slot must belong to one dequant group");
 static_assert(kPairRingC % kPairDeqGroups == 0, "each code slot must belong to one dequant group");
 constexpr int kPairDeqWarps = 4;                 // warps per group (128 weight rows)
-constexpr int kPairThreads = 64 + kPairDeqGroups * kPairDeqWarps * 32;
+constexpr int kPairIssuers = 2;
+static_assert(kPairRingA % kPairIssuers == 0 && kPairRingW % kPairIssuers == 0, "each operand slot must belong to one issuer");
+constexpr int kPairIssuerWarp1 = 2 + kPairDeqGroups * kPairDeqWarps;   // second MMA issuer
+constexpr int kPairThreads = 64 + kPairDeqGroups * kPairDeqWarps * 32 + 32;
 constexpr uint32_t kPairABytes = 128 * 64 * 2;   // 16 KB activations (this CTA's half)
 constexpr uint32_t kPairWBytes = 128 * 64 * 2;   // 16 KB dequantised weight half
 constexpr uint32_t kPairCBytes = 128 * 64 / 2;   //  4 KB packed codes
@@ -55,7 +63,7 @@ constexpr uint32_t kPairOffW = kPairRingA * kPairABytes;
 constexpr uint32_t kPairOffC = kPairOffW + kPairRingW * kPairWBytes;
 constexpr uint32_t kPairOffBar = kPairOffC + kPairRingC * kPairCBytes;
 constexpr uint32_t kPairSmemBytes = kPairOffBar + 1024 /*align*/ + 512 /*bars*/ + 4 * kPairDeqGroups * 128;
-constexpr uint32_t kPairTmemCols = 256;
+constexpr uint32_t kPairTmemCols = 512;   // D0 (even stages) at 0, D1 (odd stages) at 256
 static_assert(kPairSmemBytes <= 227 * 1024, "pair kernel shared memory");
 
 template <int MODE>
@@ -102,7 +110,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       mbar_init(smem_u32(&full_w[i]), 2 * kPairDeqWarps);
       mbar_init(smem_u32(&empty_w[i]), 1);
     }
-    mbar_init(smem_u32(acc_full), 1);
+    mbar_init(smem_u32(acc_full), kPairIssuers);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -185,11 +193,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------- MMA issuer (leader)
+  } else if (warp == 1 || warp == kPairIssuerWarp1) {
+    // ------------------------------------------------- MMA issuers (leader)
     if (leader && lane == 0) {
+      const int me = (warp == 1) ? 0 : 1;
+      const uint32_t dcol = tmem_d + 256u * me;
       constexpr uint32_t idesc = idesc_bf16(256, 256, 0, MODE == kModeDx ? 1 : 0);
-      for (int it = 0; it < total; ++it) {
+      for (int it = me; it < total; it += kPairIssuers) {
         const int ia = it % kPairRingA, iw = it % kPairRingW;
         if (!mbar_wait(smem_u32(&full_a[ia]), par(it, kPairRingA), abort_flag, args.status)) break;
         if (!mbar_wait(smem_u32(&full_w[iw]), par(it, kPairRingW), abort_flag, args.status)) break;
@@ -201,7 +211,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const uint64_t adesc = sw128_desc(a_base + k * 32, 16, 1024);
           const uint64_t bdesc = (MODE == kModeFwd) ? sw128_desc(w_base + k * 32, 16, 1024)
                                                     : sw128_desc(w_base + k * 2048, 8192, 1024);
-          umma_bf16_pair(tmem_d, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
+          umma_bf16_pair(dcol, adesc, bdesc, idesc, (it > me || k > 0) ? 1u : 0u);
         }
         umma_commit_pair(smem_u32(&empty_a[ia]), 0x3);
         umma_commit_pair(smem_u32(&empty_w[iw]), 0x3);
@@ -335,9 +345,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll 1
       for (int c = g; c < 16; c += kPairDeqGroups) {
         const int col = c * 16;
-        uint32_t r[16];
+        uint32_t r[16], r1[16];
         tmem_ld16(taddr + col, r);
+        tmem_ld16(taddr + 256 + col, r1);
         tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r1[i]));
         const int64_t gc = np0 + col;
         if (row < args.M && gc < args.out_cols) {
           uint32_t pk[8];
