@@ -45,6 +45,12 @@ L2_BYTES = 126 * 1024 * 1024
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM traffic of one fused-GEMM launch (gate forward) from the ncu capture
+# summarised in profiles/k_gemm_nf4_pair_fwd_gate_m2048.md; None once the
+# kernel changes and until it is captured again.
+GEMM_TRAFFIC_BYTES = 48.93e6
+
+
 def step_flops(wl=WL, M=None) -> float:
     M = wl.M if M is None else M
     return float(sum(4 * M * N * K + 6 * M * wl.r * (N + K) for _, N, K in wl.shapes))
@@ -350,13 +356,19 @@ def run_ours(args):
                    "weights": "NF4 double-quant, block 64, group 256",
                    "flops_per_step": step_flops(), "l2": "flushed between timed steps",
                    "parallelism": f"dp{world}"},
-        "roofline": {"bound": "tensor", "kernel": "k_gemm_nf4 (fused NF4 dequant + tcgen05 GEMM)",
+        "roofline": {"bound": "tensor", "kernel": "k_gemm_nf4_pair (fused NF4 dequant + 2-SM tcgen05 GEMM)",
                      "achieved": round(g_achieved, 2), "peak": round(peak_sus, 1), "unit": "TFLOP/s",
                      "frac": round(g_achieved / peak_sus, 4),
                      "peak_source": f"{peaks_src} bf16_tflops_sustained",
                      "frac_of_burst_peak": round(g_achieved / peak_burst, 4),
                      "launches": g_launches, "avg_launch_us": round(g_time / g_launches * 1e6, 2),
-                     "share_of_step": round(gemm_share, 4), "traffic": None},
+                     "share_of_step": round(gemm_share, 4),
+                     # DRAM bytes (read + write) of one launch, from the ncu capture in
+                     # profiles/k_gemm_nf4_pair_fwd_gate_m2048.md (gate forward,
+                     # 2048 x 11008 x 4096); its algorithmic bytes are 85.1 MB, most of
+                     # Y still sitting in L2 at the end of the kernel
+                     "traffic": GEMM_TRAFFIC_BYTES, "traffic_launch": "gate fwd, M 2048 x N 11008 x K 4096",
+                     "traffic_algorithmic": 85.1e6},
         "gpu_launches": launches_per_step(WL) * args.steps,
         "clocks": clk,
         "e2e": e2e,
