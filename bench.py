@@ -222,7 +222,11 @@ def run_ours(args):
     layer = Layer(q, WL, WL.M, dev, rank)
     layer.quantize_all()
     torch.cuda.synchronize()
+    # a short device-side spin first, so that all 7 launches are queued before
+    # the first event: the events then time the kernels, not the host's
+    # launch gaps (each Python call takes longer to issue than its kernel runs)
     qev = []
+    torch.cuda._sleep(2_000_000)
     layer.quantize_all(events=qev)
     torch.cuda.synchronize()
     quant_ms = sum(a.elapsed_time(b) for a, b in qev)
@@ -394,6 +398,120 @@ def time_events(fn, reps, flush=None):
     return [a.elapsed_time(b) for a, b in evs]
 
 
+def _quantize_model(q, wl, dev, status):
+    """Generate every weight of workload `wl` on the device one matrix at a
+    time, quantise it into resident NF4 storage and free the bf16 source.
+    Returns (nf4 weights [layer][projection], quantiser kernel ms, params)."""
+    nf4, evs, params = [], [], 0
+    for L in range(wl.layers):
+        row = []
+        for i, (name, N, K) in enumerate(wl.shapes):
+            W = inputs.weight((N, K), wl.w_std, inputs.matrix_seed(wl.base_seed, L, i), device=dev)
+            Wq = q.empty_nf4(N, K, dev)
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev[0].record()
+            q.qlora_quantize_nf4(W, out=Wq, d_status=status)
+            ev[1].record()
+            evs.append(ev)
+            del W
+            row.append(Wq)
+            params += N * K
+        nf4.append(row)
+    torch.cuda.synchronize()
+    return nf4, sum(a.elapsed_time(b) for a, b in evs), params
+
+
+def _layer_tensors(wl, L, M, dev, x_shared=True):
+    """Adapters and activations of one layer.  With x_shared, q/k/v read one
+    input and gate/up another, as in a LLaMA decoder layer."""
+    xkey = {0: 0, 1: 0, 2: 0, 3: 3, 4: 4, 5: 4, 6: 6} if x_shared else {i: i for i in range(7)}
+    xs, out = {}, []
+    for i, (name, N, K) in enumerate(wl.shapes):
+        seed = inputs.matrix_seed(wl.base_seed, L, i)
+        k = xkey[i]
+        if k not in xs:
+            xs[k] = inputs.normal((M, K), 1.0, inputs.matrix_seed(wl.base_seed, L, k) * 16 + 1, dev)
+        out.append(dict(X=xs[k], dY=inputs.normal((M, N), 1.0, seed * 16 + 2, dev),
+                        A=inputs.normal((wl.r, K), 0.01, seed * 16 + 3, dev),
+                        B=inputs.normal((N, wl.r), 0.01, seed * 16 + 4, dev),
+                        T=torch.empty((M, wl.r), dtype=torch.float32, device=dev),
+                        dA=torch.empty((wl.r, K), dtype=torch.float32, device=dev),
+                        dB=torch.empty((N, wl.r), dtype=torch.float32, device=dev)))
+    return out
+
+
+def _model_step(q, wl, nf4, acts, bufs, ws, status, layers):
+    """Forward through every projection of `layers`, then backward in reverse."""
+    for L in layers:
+        for i in range(len(wl.shapes)):
+            a = acts[L][i]
+            q.qlora_linear_fwd(a["X"], nf4[L][i], a["A"], a["B"], wl.alpha, Y=bufs[i]["Y"], T_save=a["T"],
+                               workspace=ws, d_status=status)
+    for L in reversed(layers):
+        for i in reversed(range(len(wl.shapes))):
+            a = acts[L][i]
+            q.qlora_linear_bwd(a["dY"], a["X"], nf4[L][i], a["A"], a["B"], wl.alpha, T_saved=a["T"],
+                               dX=bufs[i]["dX"], dA=a["dA"], dB=a["dB"], workspace=ws, d_status=status)
+
+
+def _time_model_step(q, wl, nf4, acts, M, dev, layers, steps, warmup):
+    bufs = [dict(Y=torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+                 dX=torch.empty((M, K), dtype=torch.bfloat16, device=dev)) for (_, N, K) in wl.shapes]
+    ws = torch.empty(max(q.qlora_workspace_bytes(M, N, K, wl.r) for (_, N, K) in wl.shapes),
+                     dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(warmup):
+        _model_step(q, wl, nf4, acts, bufs, ws, status, layers)
+    torch.cuda.synchronize()
+    ms = time_events(lambda: _model_step(q, wl, nf4, acts, bufs, ws, status, layers), steps)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device status set during a config workload"
+    t = statistics.median(ms)
+    flops = len(layers) * step_flops(wl, M)
+    return {"value": round(flops / (t * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(t, 3),
+            "tokens": M, "layers": len(layers), "flops_per_step": flops, "steps": steps, "warmup": warmup}
+
+
+def config_workloads(q, dev, hbm):
+    """The 32-layer 7B stack and the 80-layer 65B model: whole-model one-shot
+    quantisation on the GPU, then training steps through the resident NF4
+    weights (all 224 projections at 4096 tokens; one 65B layer at 8192)."""
+    out = {}
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    # 32-layer LLaMA-7B-shaped stack, 4096 tokens, r = 16
+    wl = inputs.STACK7B
+    nf4, qms, params = _quantize_model(q, wl, dev, status)
+    qbytes = params * (2 + 0.5 + 1 / 64 + 4 / 16384)
+    acts = [_layer_tensors(wl, L, wl.M, dev) for L in range(wl.layers)]
+    torch.cuda.synchronize()
+    step = _time_model_step(q, wl, nf4, acts, wl.M, dev, list(range(wl.layers)), steps=2, warmup=1)
+    out["stack7b_32layer"] = {
+        "quantize": {"params": params, "ms": round(qms, 3), "value": round(qbytes / (qms * 1e-3) / 1e9, 1),
+                     "unit": "GB/s (bf16 in + NF4 out)", "frac_of_hbm": round(qbytes / (qms * 1e-3) / 1e9 / hbm, 4),
+                     "nf4_resident_gb": round(sum(w.nbytes() for row in nf4 for w in row) / 1e9, 3)},
+        "step": step}
+    del nf4, acts
+    torch.cuda.empty_cache()
+    # 80-layer LLaMA-65B-shaped model: all weights quantised and resident,
+    # then one layer's 7 projections at 8192 tokens, r = 64
+    wl = inputs.LLAMA65B
+    nf4, qms, params = _quantize_model(q, wl, dev, status)
+    qbytes = params * (2 + 0.5 + 1 / 64 + 4 / 16384)
+    resident = sum(w.nbytes() for row in nf4 for w in row)
+    acts = {0: _layer_tensors(wl, 0, wl.M, dev)}
+    torch.cuda.synchronize()
+    step = _time_model_step(q, wl, nf4, acts, wl.M, dev, [0], steps=3, warmup=2)
+    assert int(status.item()) == 0
+    out["llama65b_80layer"] = {
+        "quantize": {"params": params, "ms": round(qms, 3), "value": round(qbytes / (qms * 1e-3) / 1e9, 1),
+                     "unit": "GB/s (bf16 in + NF4 out)", "frac_of_hbm": round(qbytes / (qms * 1e-3) / 1e9 / hbm, 4),
+                     "nf4_resident_gb": round(resident / 1e9, 3)},
+        "layer_step": step}
+    del nf4, acts
+    torch.cuda.empty_cache()
+    return out
+
+
 def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_params):
     hbm = float(peaks["hbm_gbs"])
     out = {}
@@ -441,7 +559,10 @@ def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_param
             for _ in range(3):
                 fn()
             it = iter(kev)
-            ms = statistics.median(time_events(fn, 10, flush=lambda: l2buf.add_(1)))
+            # the flush is followed by a device-side spin so that the call's
+            # launches are queued before its start event: the whole-call time
+            # is GPU time, not host launch gaps
+            ms = statistics.median(time_events(fn, 10, flush=lambda: (l2buf.add_(1), torch.cuda._sleep(400_000))))
             kms = statistics.median(a.elapsed_time(b) for a, b in kev)
             wbytes = Wq.nbytes()
             res.append({"matrix": [N, K], "us": round(ms * 1e3, 2),
@@ -456,6 +577,9 @@ def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_param
                         "kernel_frac_of_hbm": round(sum(kgbs) / len(kgbs) / hbm, 4)}
     out["decode_gemv"] = {"unit": "GB/s of NF4 weight (121.17 MB per matrix)", **dec,
                           "peak_hbm_gbs": hbm}
+    del mats
+    torch.cuda.empty_cache()
+    out.update(config_workloads(q, dev, hbm))
     return out
 
 

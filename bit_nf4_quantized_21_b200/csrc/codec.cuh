@@ -35,9 +35,10 @@ __device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
 }
 
 // Nearest NF4 level of a normalised weight: code = #{i : x > t_i}, found by a
-// 4-step binary search over the 15 sorted thresholds held in shared memory.
-__device__ __forceinline__ uint32_t nf4_encode(float x, const float* s_thr) {
-  uint32_t c = (x > s_thr[7]) ? 8u : 0u;
+// 4-step binary search over the 15 sorted thresholds; the first step's
+// threshold (t_7) comes from a register, the other three from shared memory.
+__device__ __forceinline__ uint32_t nf4_encode(float x, const float* s_thr, float t7) {
+  uint32_t c = (x > t7) ? 8u : 0u;
   c += (x > s_thr[c + 3]) ? 4u : 0u;
   c += (x > s_thr[c + 1]) ? 2u : 0u;
   c += (x > s_thr[c]) ? 1u : 0u;
@@ -48,6 +49,8 @@ __device__ __forceinline__ uint32_t nf4_encode(float x, const float* s_thr) {
 // share a 64-weight block (8 weights each, one 16-byte load of bf16), so a
 // warp reads 4 whole blocks = 512 contiguous bytes and writes 128 contiguous
 // bytes of codes.  The block absmax is a warp-shuffle max over the 8 lanes.
+// All 8 of a thread's loads are issued before any is used, so every thread
+// keeps 8 x 16 B in flight (HBM needs tens of KB per SM in flight).
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
     k_quantize_nf4(const T* __restrict__ w, int64_t nblocks, int dq, uint8_t* __restrict__ codes,
@@ -64,19 +67,24 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int64_t b0 = g * 256;
   const int nb = static_cast<int>((nblocks - b0) < 256 ? (nblocks - b0) : 256);
   const int sub = tid & 7;
+  const float t7 = c_nf4_threshold[7];
   bool nonfinite = false;
 
-#pragma unroll 1
+  float v[8][8];
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int lb = it * 32 + (tid >> 3);
+    if (lb < nb) load8<T>(w + (b0 + lb) * 64 + sub * 8, v[it]);
+  }
+#pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int lb = it * 32 + (tid >> 3);
     const bool valid = lb < nb;
     const int64_t b = b0 + lb;
-    float v[8];
     uint32_t mbits = 0;
     if (valid) {
-      load8<T>(w + b * 64 + sub * 8, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mbits = max(mbits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+      for (int i = 0; i < 8; ++i) mbits = max(mbits, __float_as_uint(v[it][i]) & 0x7FFFFFFFu);
     }
     // max over the 8 lanes of the block (integer order = magnitude order,
     // with inf/NaN patterns above every finite value)
@@ -93,7 +101,7 @@ __global__ void __launch_bounds__(kQuantThreads)
       const float inv = __frcp_rn(absmax);
       word = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) word |= nf4_encode(__fmul_rn(v[i], inv), s_thr) << (4 * i);
+      for (int i = 0; i < 8; ++i) word |= nf4_encode(__fmul_rn(v[it][i], inv), s_thr, t7) << (4 * i);
     }
     reinterpret_cast<uint32_t*>(codes)[b * 8 + sub] = word;
     if (sub == 0) s_absmax[lb] = absmax;

@@ -204,15 +204,17 @@ def linear_fwd(X, W_hat, A, B, alpha: float, r: int):
 
 def linear_bwd(dY, X, W_hat, A, B, alpha: float, r: int, T=None):
     """Returns dict(dX, dA, dB, G) in binary64.  T is recomputed as X A^T when
-    not given."""
-    dY, X, W, A, B = _f64(dY), _f64(X), _f64(W_hat), _f64(A), _f64(B)
+    not given.  W_hat = None skips dX (returned as None): dA and dB need only
+    the rank-r products, so they can be checked over many more tokens than
+    the M x N x K product allows."""
+    dY, X, A, B = _f64(dY), _f64(X), _f64(A), _f64(B)
     s = float(alpha) / float(r)
     if T is None:
         T = X @ A.T
     else:
         T = np.asarray(T, np.float64)
     G = dY @ B
-    dX = dY @ W + s * (G @ A)
+    dX = None if W_hat is None else dY @ _f64(W_hat) + s * (G @ A)
     dA = s * (G.T @ X)
     dB = s * (dY.T @ T)
     return {"dX": dX, "dA": dA, "dB": dB, "G": G, "T": T}
