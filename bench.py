@@ -191,10 +191,11 @@ def flush_l2(buf):
 
 
 def launches_per_step(wl) -> int:
-    # forward: T skinny + finish + GEMM; backward: G skinny + finish + dX GEMM +
-    # T split + dA skinny + finish + dB skinny + finish (+1 pad each when r % 8)
+    # this library's kernels per projection: forward T skinny + fused GEMM;
+    # backward G skinny (+ T planes) + dX GEMM + one dA/dB skinny (+1 pad of
+    # B when r % 8).  The counter clears are memset nodes, not kernels.
     pad = 1 if wl.r % 8 else 0
-    return len(wl.shapes) * (3 + 8 + 2 * pad)
+    return len(wl.shapes) * (2 + 3 + pad)
 
 
 def run_ours(args):

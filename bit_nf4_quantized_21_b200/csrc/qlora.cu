@@ -133,15 +133,23 @@ struct SkPlan {
   int64_t P;
   int64_t Qtot;
   int Qn;
+  int ptiles;
   int qchunks;
   int num_chunks;
   int splits;
   int per_split;
   int stages;
   size_t partial_bytes;
+  int ctas() const { return ptiles * splits * qchunks; }
 };
 
-SkPlan plan_skinny(int64_t P, int64_t J, int64_t Qtot) {
+// Split the contraction so that the launch has at most `target` CTAs (one
+// wave: a CTA's fixed cost -- TMEM, pipeline fill, epilogue -- is a large
+// part of its time, so a second, partly filled round of CTAs nearly doubles
+// the kernel), or exactly `force_splits` splits when given.  Fewer splits
+// also mean less fp32 partial traffic (written, then re-read by the CTA that
+// finishes the tile).
+SkPlan plan_skinny(int64_t P, int64_t J, int64_t Qtot, int64_t target = 148, int64_t force_splits = 0) {
   SkPlan pl{};
   pl.P = P;
   pl.Qtot = Qtot;
@@ -149,14 +157,14 @@ SkPlan plan_skinny(int64_t P, int64_t J, int64_t Qtot) {
   pl.qchunks = static_cast<int>(cdiv(Qtot, 256));
   pl.num_chunks = static_cast<int>(cdiv(J, 64));
   const int64_t ptiles = cdiv(P, kSkBM);
-  const int64_t target = 2 * 148;
-  int64_t splits = cdiv(target, ptiles * pl.qchunks);
+  pl.ptiles = static_cast<int>(ptiles);
+  int64_t splits = force_splits > 0 ? force_splits : target / (ptiles * pl.qchunks);
   splits = std::max<int64_t>(1, std::min<int64_t>(splits, std::max(1, pl.num_chunks / 2)));
   pl.per_split = static_cast<int>(cdiv(pl.num_chunks, splits));
   pl.splits = static_cast<int>(cdiv(pl.num_chunks, pl.per_split));
   const uint32_t stage_bytes = kSkABytes + static_cast<uint32_t>(pl.Qn) * 128u;
   pl.stages = static_cast<int>(std::max<uint32_t>(2, std::min<uint32_t>(6, (200u * 1024u) / stage_bytes)));
-  pl.partial_bytes = static_cast<size_t>(pl.splits) * P * Qtot * 4;
+  pl.partial_bytes = (pl.splits * pl.qchunks > 1) ? static_cast<size_t>(pl.splits) * P * Qtot * 4 : 0;
   return pl;
 }
 
@@ -164,9 +172,14 @@ size_t skinny_smem(const SkPlan& pl) {
   return static_cast<size_t>(pl.stages) * (kSkABytes + pl.Qn * 128u) + 1024 + 256;
 }
 
-template <int A_MN, int B_MN>
-qlora_status launch_skinny(const SkPlan& pl, const CUtensorMap& ta, const CUtensorMap& tb, float* partial,
-                           int* status, cudaStream_t st) {
+// One adapter product: its plan, operand tensor maps and arguments.
+struct SkJob {
+  SkPlan pl;
+  CUtensorMap ta, tb;
+  SkinnyArgs a;
+};
+
+SkinnyArgs sk_args(const SkPlan& pl, float* partial, unsigned int* cnt, int* status) {
   SkinnyArgs a{};
   a.P = pl.P;
   a.Qn = pl.Qn;
@@ -174,16 +187,31 @@ qlora_status launch_skinny(const SkPlan& pl, const CUtensorMap& ta, const CUtens
   a.num_chunks = pl.num_chunks;
   a.chunks_per_split = pl.per_split;
   a.stages = pl.stages;
+  a.ptiles = pl.ptiles;
+  a.splits = pl.splits;
+  a.qchunks = pl.qchunks;
   a.partial = partial;
+  a.cnt = cnt;
   a.status = status;
-  dim3 grid(static_cast<unsigned>(cdiv(pl.P, kSkBM)), pl.splits, pl.qchunks);
-  k_skinny<A_MN, B_MN><<<grid, kSkThreads, skinny_smem(pl), st>>>(ta, tb, a);
+  return a;
+}
+
+// One launch for one job, or for two independent jobs of the same operand
+// majorness (CTAs [0, n0) run j0, the rest j1).
+template <int A_MN, int B_MN>
+qlora_status launch_skinny(const SkJob& j0, const SkJob* j1, cudaStream_t st) {
+  const int n0 = j0.pl.ctas();
+  const int n1 = j1 ? j1->pl.ctas() : 0;
+  const size_t smem = std::max(skinny_smem(j0.pl), j1 ? skinny_smem(j1->pl) : size_t(0));
+  const SkJob& o = j1 ? *j1 : j0;
+  k_skinny<A_MN, B_MN><<<static_cast<unsigned>(n0 + n1), kSkThreads, smem, st>>>(j0.ta, j0.tb, o.ta, o.tb, j0.a,
+                                                                                 o.a, n0);
   return check_launch();
 }
 
 // -------------------------------------------------------- workspace layout
 struct Ws {
-  size_t partial, t32, sx, ghl, thl, bpad, gv_part, gv_cnt, total;
+  size_t partial, partial2, cnt, t32, sx, ghl, thl, bpad, gv_part, gv_cnt, total;
 };
 
 // Token counts up to this take the weight-streaming decode kernel.
@@ -204,16 +232,36 @@ Dims dims_of(int64_t M, int64_t N, int64_t K, int r) {
   return d;
 }
 
+// Skinny plans of one layer call (dA and dB share one launch).
+struct SkPlans {
+  SkPlan T, G, dA, dB;
+};
+SkPlans plans_of(const Dims& d) {
+  SkPlans p;
+  p.T = plan_skinny(d.M, d.K, d.r16);
+  p.G = plan_skinny(d.M, d.N, d.r64);
+  // dA and dB share one launch: one split count for both, so that together
+  // they fill (at most) one wave
+  const int64_t qc = cdiv(d.Qh, 256);
+  const int64_t pt = (cdiv(d.K, kSkBM) + cdiv(d.N, kSkBM)) * qc;
+  const int64_t sp = std::max<int64_t>(1, 148 / pt);
+  p.dA = plan_skinny(d.K, d.M, d.Qh, 0, sp);
+  p.dB = plan_skinny(d.N, d.M, d.Qh, 0, sp);
+  return p;
+}
+// Arrival counters: T, G, dA, dB tiles, one 32-bit word each.
+size_t cnt_words(const SkPlans& p) { return p.T.ptiles + p.G.ptiles + p.dA.ptiles + p.dB.ptiles; }
+
 Ws ws_layout(const Dims& d) {
-  size_t part = 0;
-  part = std::max(part, plan_skinny(d.M, d.K, d.r16).partial_bytes);   // T
-  part = std::max(part, plan_skinny(d.M, d.N, d.r64).partial_bytes);   // G
-  part = std::max(part, plan_skinny(d.K, d.M, d.Qh).partial_bytes);    // dA
-  part = std::max(part, plan_skinny(d.N, d.M, d.Qh).partial_bytes);    // dB
+  const SkPlans pl = plans_of(d);
   auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
   Ws w{};
   size_t off = 0;
-  w.partial = off; off += a256(part);
+  // T and G run alone; dA and dB run side by side in one launch
+  w.partial = off;
+  w.partial2 = off + a256(pl.dA.partial_bytes);
+  off += a256(std::max({pl.T.partial_bytes, pl.G.partial_bytes, a256(pl.dA.partial_bytes) + pl.dB.partial_bytes}));
+  w.cnt = off; off += a256(cnt_words(pl) * 4);
   w.t32 = off; off += a256(static_cast<size_t>(d.M) * d.r * 4);
   w.sx = off; off += a256(static_cast<size_t>(2 * d.M) * d.r8 * 2);
   w.ghl = off; off += a256(static_cast<size_t>(d.M) * d.Qh * 2);
@@ -241,27 +289,35 @@ qlora_status check_linear(int64_t M, const qlora_nf4_weight* Wq, int r, float al
   return QLORA_OK;
 }
 
-// Finish a token-indexed skinny result (T or G).
-qlora_status finish_rows(const float* src, int64_t src_ld, int splits, int64_t split_stride, const Dims& d,
-                         float s, float* f32, __nv_bfloat16* s_bf16, __nv_bfloat16* hl, cudaStream_t st) {
-  const int width = std::max(d.r16, d.Qh - 2 * d.r16);
-  const int64_t n = d.M * width;
-  k_finish_rows<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, st>>>(src, src_ld, splits, split_stride, d.M, d.r,
-                                                                     d.r8, d.r16, d.Qh, s, f32, s_bf16, hl);
-  return check_launch();
+// The final transform of a token-indexed product (T or G) into `a`.
+void sk_rows(SkinnyArgs& a, const Dims& d, float s, float* f32, __nv_bfloat16* s_bf16, __nv_bfloat16* hl) {
+  a.finish = kFinRows;
+  a.s = s; a.r = d.r; a.r8 = d.r8; a.r16 = d.r16; a.Qh = d.Qh;
+  a.f32 = f32; a.s_bf16 = s_bf16; a.hl = hl;
+}
+// Counter words of T, G, dA, dB inside the workspace's counter region.
+unsigned int* cnt_T(uint8_t* ws, const Ws& L) { return reinterpret_cast<unsigned int*>(ws + L.cnt); }
+unsigned int* cnt_G(uint8_t* ws, const Ws& L, const SkPlans& p) { return cnt_T(ws, L) + p.T.ptiles; }
+unsigned int* cnt_dA(uint8_t* ws, const Ws& L, const SkPlans& p) { return cnt_G(ws, L, p) + p.G.ptiles; }
+unsigned int* cnt_dB(uint8_t* ws, const Ws& L, const SkPlans& p) { return cnt_dA(ws, L, p) + p.dA.ptiles; }
+
+// Clear the arrival counters of one call (they must start at zero).
+qlora_status clear_counters(uint8_t* ws, const Ws& L, const SkPlans& p, cudaStream_t st) {
+  return cudaMemsetAsync(ws + L.cnt, 0, cnt_words(p) * 4, st) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-// T = X A^T  (fp32 into t32, and optionally s*T in bf16 into sx).
+// T = X A^T  (fp32 into t32, and optionally s*T in bf16 planes into sx), one
+// launch.  The caller has cleared the counters.
 qlora_status run_T(const void* X, const void* A, const Dims& d, float s, uint8_t* ws, const Ws& L, float* t32,
                    __nv_bfloat16* sx, int* status, cudaStream_t st) {
-  SkPlan pl = plan_skinny(d.M, d.K, d.r16);
-  CUtensorMap ta, tb;
-  if (!bf16_map(&ta, X, d.K, d.M, d.K, 64, kSkBM)) return QLORA_ERR_CUDA;
-  if (!bf16_map(&tb, A, d.K, d.r, d.K, 64, static_cast<uint32_t>(pl.Qn))) return QLORA_ERR_CUDA;
-  float* partial = reinterpret_cast<float*>(ws + L.partial);
-  qlora_status rc = launch_skinny<0, 0>(pl, ta, tb, partial, status, st);
-  if (rc != QLORA_OK) return rc;
-  return finish_rows(partial, pl.Qtot, pl.splits, pl.P * pl.Qtot, d, s, t32, sx, nullptr, st);
+  const SkPlans P = plans_of(d);
+  SkJob j;
+  j.pl = P.T;
+  if (!bf16_map(&j.ta, X, d.K, d.M, d.K, 64, kSkBM)) return QLORA_ERR_CUDA;
+  if (!bf16_map(&j.tb, A, d.K, d.r, d.K, 64, static_cast<uint32_t>(j.pl.Qn))) return QLORA_ERR_CUDA;
+  j.a = sk_args(j.pl, reinterpret_cast<float*>(ws + L.partial), cnt_T(ws, L), status);
+  sk_rows(j.a, d, s, t32, sx, nullptr);
+  return launch_skinny<0, 0>(j, nullptr, st);
 }
 
 const void* padded_B(const void* B, const Dims& d, uint8_t* ws, const Ws& L, cudaStream_t st, qlora_status* rc) {
@@ -493,12 +549,16 @@ qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* 
 
   if (M <= kDecodeMaxM) {
     // decode shape: T = X A^T (fp32), then the weight-streaming kernel
+    st = clear_counters(ws, L, plans_of(d), cs);
+    if (st != QLORA_OK) return st;
     st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
     if (st != QLORA_OK) return st;
     return run_gemv(X, Wq, d, t32, B, Y, s, ws, L, events, d_status, cs);
   }
 
   // 1. T = X A^T and s*T (bf16) for the fold
+  st = clear_counters(ws, L, plans_of(d), cs);
+  if (st != QLORA_OK) return st;
   st = run_T(X, A, d, s, ws, L, t32, sT, d_status, cs);
   if (st != QLORA_OK) return st;
   const void* Bp = padded_B(B, d, ws, L, cs, &st);
@@ -525,23 +585,36 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
   const Ws L = ws_layout(d);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const float s = alpha / static_cast<float>(r);
-  float* partial = reinterpret_cast<float*>(ws + L.partial);
+  const SkPlans P = plans_of(d);
   __nv_bfloat16* sG = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
   __nv_bfloat16* Ghl = reinterpret_cast<__nv_bfloat16*>(ws + L.ghl);
   __nv_bfloat16* Thl = reinterpret_cast<__nv_bfloat16*>(ws + L.thl);
 
   const void* Bp = padded_B(B, d, ws, L, cs, &st);
   if (st != QLORA_OK) return st;
-
-  // 1. G = dY B -> s*G (bf16, for the dX fold) and [G_hi | G_lo] (for dA)
-  {
-    SkPlan pl = plan_skinny(d.M, d.N, d.r64);
-    CUtensorMap ta, tb;
-    if (!bf16_map(&ta, dY, d.N, d.M, d.N, 64, kSkBM)) return QLORA_ERR_CUDA;
-    if (!bf16_map(&tb, Bp, d.r8, d.N, d.r8, 64, 64)) return QLORA_ERR_CUDA;
-    st = launch_skinny<0, 1>(pl, ta, tb, partial, d_status, cs);
+  st = clear_counters(ws, L, P, cs);
+  if (st != QLORA_OK) return st;
+  // 0. T recomputed when the forward's was not kept
+  const float* t = T_saved;
+  if (!t) {
+    float* t32 = reinterpret_cast<float*>(ws + L.t32);
+    st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
     if (st != QLORA_OK) return st;
-    st = finish_rows(partial, pl.Qtot, pl.splits, pl.P * pl.Qtot, d, s, nullptr, sG, Ghl, cs);
+    t = t32;
+  }
+  // 1. G = dY B -> s*G (bf16 planes, for the dX fold) and [G_hi | G_lo] (for
+  //    dA); the same launch turns T into [T_hi | T_lo] (for dB)
+  {
+    SkJob j;
+    j.pl = P.G;
+    if (!bf16_map(&j.ta, dY, d.N, d.M, d.N, 64, kSkBM)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&j.tb, Bp, d.r8, d.N, d.r8, 64, 64)) return QLORA_ERR_CUDA;
+    j.a = sk_args(j.pl, reinterpret_cast<float*>(ws + L.partial), cnt_G(ws, L, P), d_status);
+    sk_rows(j.a, d, s, nullptr, sG, Ghl);
+    j.a.side_src = t;
+    j.a.side_rows = d.M;
+    j.a.side_hl = Thl;
+    st = launch_skinny<0, 1>(j, nullptr, cs);
     if (st != QLORA_OK) return st;
   }
   // 2. dX = dY W^ + (sG) A
@@ -549,43 +622,29 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
     st = run_fused(kModeDx, dY, Wq, d, sG, A, dX, events, d_status, cs);
     if (st != QLORA_OK) return st;
   }
-  // 3. T (saved or recomputed) -> [T_hi | T_lo]
+  // 3. dA = s G^T X (C[k, q] = sum_m X[m, k] Ghl[m, q]) and dB = s dY^T T
+  //    (C[n, q] = sum_m dY[m, n] Thl[m, q]) in one launch
   {
-    const float* t = T_saved;
-    if (!t) {
-      float* t32 = reinterpret_cast<float*>(ws + L.t32);
-      st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
-      if (st != QLORA_OK) return st;
-      t = t32;
+    const int out_bf16 = grad_dtype == QLORA_BF16 ? 1 : 0;
+    SkJob ja, jb;
+    ja.pl = P.dA;
+    jb.pl = P.dB;
+    if (!bf16_map(&ja.ta, X, d.K, d.M, d.K, 64, 64)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&ja.tb, Ghl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&jb.ta, dY, d.N, d.M, d.N, 64, 64)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&jb.tb, Thl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
+    ja.a = sk_args(ja.pl, reinterpret_cast<float*>(ws + L.partial), cnt_dA(ws, L, P), d_status);
+    jb.a = sk_args(jb.pl, reinterpret_cast<float*>(ws + L.partial2), cnt_dB(ws, L, P), d_status);
+    for (SkinnyArgs* a : {&ja.a, &jb.a}) {
+      a->finish = kFinGrad;
+      a->s = s; a->r = d.r; a->r8 = d.r8; a->r16 = d.r16; a->Qh = d.Qh;
+      a->out_bf16 = out_bf16;
     }
-    st = finish_rows(t, d.r, 1, 0, d, s, nullptr, nullptr, Thl, cs);
-    if (st != QLORA_OK) return st;
-  }
-  const int out_bf16 = grad_dtype == QLORA_BF16 ? 1 : 0;
-  // 4. dA = s G^T X   (C[k, q] = sum_m X[m, k] Ghl[m, q])
-  {
-    SkPlan pl = plan_skinny(d.K, d.M, d.Qh);
-    CUtensorMap ta, tb;
-    if (!bf16_map(&ta, X, d.K, d.M, d.K, 64, 64)) return QLORA_ERR_CUDA;
-    if (!bf16_map(&tb, Ghl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
-    st = launch_skinny<1, 1>(pl, ta, tb, partial, d_status, cs);
-    if (st != QLORA_OK) return st;
-    dim3 g(static_cast<unsigned>(cdiv(d.K, 32)), static_cast<unsigned>(cdiv(d.r, 32)));
-    k_finish_grad<<<g, 256, 0, cs>>>(partial, pl.Qtot, pl.splits, d.K, d.r, d.r16, s, 1, out_bf16, dA);
-    st = check_launch();
-    if (st != QLORA_OK) return st;
-  }
-  // 5. dB = s dY^T T  (C[n, q] = sum_m dY[m, n] Thl[m, q])
-  {
-    SkPlan pl = plan_skinny(d.N, d.M, d.Qh);
-    CUtensorMap ta, tb;
-    if (!bf16_map(&ta, dY, d.N, d.M, d.N, 64, 64)) return QLORA_ERR_CUDA;
-    if (!bf16_map(&tb, Thl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
-    st = launch_skinny<1, 1>(pl, ta, tb, partial, d_status, cs);
-    if (st != QLORA_OK) return st;
-    dim3 g(static_cast<unsigned>(cdiv(d.N, 32)), static_cast<unsigned>(cdiv(d.r, 32)));
-    k_finish_grad<<<g, 256, 0, cs>>>(partial, pl.Qtot, pl.splits, d.N, d.r, d.r16, s, 0, out_bf16, dB);
-    st = check_launch();
+    ja.a.transpose = 1;
+    ja.a.out = dA;
+    jb.a.transpose = 0;
+    jb.a.out = dB;
+    st = launch_skinny<1, 1>(ja, &jb, cs);
   }
   return st;
 }
@@ -618,12 +677,15 @@ qlora_status noalloc_scratch(void** out) {
   return QLORA_OK;
 }
 
-// Forward-only carve: T partials, fp32 T, s*T planes, padded B.
+// Forward-only carve: T partials, arrival counters, fp32 T, s*T planes,
+// padded B (and the decode kernel's partial tiles and counters).
 Ws noalloc_fwd_layout(const Dims& d) {
   auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
   Ws w{};
   size_t off = 0;
-  w.partial = off; off += a256(plan_skinny(d.M, d.K, d.r16).partial_bytes);
+  const SkPlans pl = plans_of(d);
+  w.partial = w.partial2 = off; off += a256(pl.T.partial_bytes);
+  w.cnt = off; off += a256(cnt_words(pl) * 4);
   w.t32 = off; off += a256(static_cast<size_t>(d.M) * d.r * 4);
   w.sx = off; off += a256(static_cast<size_t>(2 * d.M) * d.r8 * 2);
   w.ghl = w.thl = off;
@@ -662,6 +724,8 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const void* X, int64_t M, const
   float* t32 = T_save ? T_save : reinterpret_cast<float*>(ws + L.t32);
   __nv_bfloat16* sT = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
 
+  st = clear_counters(ws, L, plans_of(d), cs);
+  if (st != QLORA_OK) return st;
   if (M <= kDecodeMaxM) {
     st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
     if (st != QLORA_OK) return st;

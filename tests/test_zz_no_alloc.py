@@ -64,12 +64,14 @@ def test_noalloc_forward_matches_workspace_forward_twice(M, N, K, r):
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
-    W = inputs.weight((256, 22016), 0.02, 7, device=DEV)
+    W = inputs.weight((256, 64), 0.02, 7, device=DEV)
     Wq = q.qlora_quantize_nf4(W)
     cw = Wq.c()
-    M = 16384                                   # 64-rank forward scratch ~21 MB > 16 MiB
-    X = torch.empty((M, 22016), dtype=torch.bfloat16, device=DEV)
-    A = torch.empty((64, 22016), dtype=torch.bfloat16, device=DEV)
+    # rank 64 at M = 65536: fp32 T (16 MiB) plus the two bf16 planes of s*T
+    # (16 MiB) alone are twice the fixed scratch
+    M = 65536
+    X = torch.empty((M, 64), dtype=torch.bfloat16, device=DEV)
+    A = torch.empty((64, 64), dtype=torch.bfloat16, device=DEV)
     B = torch.empty((256, 64), dtype=torch.bfloat16, device=DEV)
     Y = torch.empty((M, 256), dtype=torch.bfloat16, device=DEV)
     rc = q.lib().qlora_linear_fwd_noalloc(X.data_ptr(), M, ctypes.byref(cw), A.data_ptr(), B.data_ptr(), 64,
