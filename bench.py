@@ -48,7 +48,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one fused-GEMM launch (gate forward) from the ncu capture
 # summarised in profiles/k_gemm_nf4_pair_fwd_gate_m2048.md; None once the
 # kernel changes and until it is captured again.
-GEMM_TRAFFIC_BYTES = 48.93e6
+GEMM_TRAFFIC_BYTES = None
 
 
 def step_flops(wl=WL, M=None) -> float:
@@ -177,6 +177,56 @@ class Layer:
             self.q.qlora_linear_bwd(p["dY"], p["X"], p["Wq"], p["A"], p["B"], alpha, T_saved=p["T"],
                                     dX=p["dX"], dA=p["dA"], dB=p["dB"], workspace=self.ws,
                                     d_status=self.status, gemm_events=ev)
+
+    def step_e2e(self, hostX, hostdY, hostdA, hostdB, s_h2d, s_d2h, ev, allreduce=None):
+        """One step from pinned host buffers: each projection's inputs are
+        copied in on s_h2d while earlier projections compute (X in forward
+        order, then dY in backward order), each projection waits only for its
+        own inputs, and its gradients go back on s_d2h as soon as its backward
+        is done.  `ev` brackets the whole step on the compute stream."""
+        q, alpha = self.q, self.wl.alpha
+        comp = torch.cuda.current_stream()
+        ev[0].record(comp)
+        s_h2d.wait_event(ev[0])
+        ready_x, ready_dy = [], {}
+        with torch.cuda.stream(s_h2d):
+            for p, hx in zip(self.proj, hostX):
+                p["X"].copy_(hx, non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(s_h2d)
+                ready_x.append(e)
+            for i in reversed(range(len(self.proj))):
+                self.proj[i]["dY"].copy_(hostdY[i], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(s_h2d)
+                ready_dy[i] = e
+        for p, e in zip(self.proj, ready_x):
+            comp.wait_event(e)
+            q.qlora_linear_fwd(p["X"], p["Wq"], p["A"], p["B"], alpha, Y=p["Y"], T_save=p["T"],
+                               workspace=self.ws, d_status=self.status)
+        done = {}
+        for i in reversed(range(len(self.proj))):
+            p = self.proj[i]
+            comp.wait_event(ready_dy[i])
+            q.qlora_linear_bwd(p["dY"], p["X"], p["Wq"], p["A"], p["B"], alpha, T_saved=p["T"],
+                               dX=p["dX"], dA=p["dA"], dB=p["dB"], workspace=self.ws, d_status=self.status)
+            e = torch.cuda.Event()
+            e.record(comp)
+            done[i] = e
+        if allreduce is not None:      # data parallel: gradients are summed first
+            allreduce()
+            e = torch.cuda.Event()
+            e.record(comp)
+            done = {i: e for i in done}
+        for i in reversed(range(len(self.proj))):
+            s_d2h.wait_event(done[i])
+            with torch.cuda.stream(s_d2h):
+                hostdA[i].copy_(self.proj[i]["dA"], non_blocking=True)
+                hostdB[i].copy_(self.proj[i]["dB"], non_blocking=True)
+        fin = torch.cuda.Event()
+        fin.record(s_d2h)
+        comp.wait_event(fin)
+        ev[1].record(comp)
 
     def gemm_flops(self):
         """Algorithmic flops of each fused-GEMM launch, in step order."""
@@ -307,20 +357,12 @@ def run_ours(args):
         d2h = sum(t.numel() * t.element_size() for t in hostdA + hostdB)
         e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(args.steps)]
+        s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
         barrier()
         torch.cuda.synchronize()
         for i in range(args.steps):
             flush_l2(l2buf)
-            e_ev[i][0].record()
-            for p, hx, hdy in zip(layer.proj, hostX, hostdY):
-                p["X"].copy_(hx, non_blocking=True)
-                p["dY"].copy_(hdy, non_blocking=True)
-            layer.step()
-            allreduce_grads()
-            for p, ha, hb in zip(layer.proj, hostdA, hostdB):
-                ha.copy_(p["dA"], non_blocking=True)
-                hb.copy_(p["dB"], non_blocking=True)
-            e_ev[i][1].record()
+            layer.step_e2e(hostX, hostdY, hostdA, hostdB, s_h2d, s_d2h, e_ev[i], allreduce_grads if world > 1 else None)
         torch.cuda.synchronize()
         barrier()
         e_ms = sum(a.elapsed_time(b) for a, b in e_ev)

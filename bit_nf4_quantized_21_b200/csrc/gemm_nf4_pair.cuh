@@ -11,9 +11,9 @@
 //
 // Three shared-memory rings per CTA; stage `it` (64 deep) uses slot
 // it % depth of each:
-//   activations  4 x 16 KB  pair TMA by producer lane 0, completing on the
-//                           leader's full_a; freed by the MMA (empty_a)
-//   codes        9 x  4 KB  local TMA by producer lane 1 (full_c); freed by
+//   activations  6 x 16 KB  pair TMA by the producer warp (0), completing on
+//                           the leader's full_a; freed by the MMA (empty_a)
+//   codes        6 x  4 KB  local TMA by the code warp (15) (full_c); freed by
 //                           the dequant warps once the codes are in
 //                           registers (empty_c)
 //   bf16 weight  6 x 16 KB  written by dequant group it % 3 after the MMA
@@ -41,8 +41,8 @@
 
 namespace qlora {
 
-constexpr int kPairRingA = 4;                    // activation ring depth
-constexpr int kPairRingC = 9;                    // packed-code ring depth
+constexpr int kPairRingA = 6;                    // activation ring depth
+constexpr int kPairRingC = 6;                    // packed-code ring depth
 constexpr int kPairRingW = 6;                    // dequantised-weight ring depth
 constexpr int kPairDeqGroups = 3;                // group it % 3 decodes stage it (owns W slots g, g + 3)
 // A waiter that takes every G-th stage must own whole slots: with a ring
@@ -55,7 +55,12 @@ constexpr int kPairDeqWarps = 4;                 // warps per group (128 weight 
 constexpr int kPairIssuers = 2;
 static_assert(kPairRingA % kPairIssuers == 0 && kPairRingW % kPairIssuers == 0, "each operand slot must belong to one issuer");
 constexpr int kPairIssuerWarp1 = 2 + kPairDeqGroups * kPairDeqWarps;   // second MMA issuer
-constexpr int kPairThreads = 64 + kPairDeqGroups * kPairDeqWarps * 32 + 32;
+// The code producer has a warp of its own: as a second lane of the
+// activation producer's warp it was starved while lane 0 spun on its ring
+// (a diverged warp runs one path at a time) and issued codes only ~half a
+// stage ahead instead of a whole ring ahead.
+constexpr int kPairCodesWarp = kPairIssuerWarp1 + 1;
+constexpr int kPairThreads = 32 * (kPairCodesWarp + 1);
 constexpr uint32_t kPairABytes = 128 * 64 * 2;   // 16 KB activations (this CTA's half)
 constexpr uint32_t kPairWBytes = 128 * 64 * 2;   // 16 KB dequantised weight half
 constexpr uint32_t kPairCBytes = 128 * 64 / 2;   //  4 KB packed codes
@@ -165,7 +170,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           while (!mbar_try_wait_cluster(fa, par(it, kPairRingA)) && global_ns() - t1 < 200000000ull) {}
         }
       }
-    } else if (lane == 1) {
+    }
+  } else if (warp == kPairCodesWarp) {
+    if (lane == 0) {
       // packed codes, freed by the dequant warps (runs ahead of the MMA)
       int issued = 0;
       for (int it = 0; it < total; ++it) {
