@@ -13,9 +13,11 @@
 // it % depth of each:
 //   activations  6 x 16 KB  pair TMA by the producer warp (0), completing on
 //                           the leader's full_a; freed by the MMA (empty_a)
-//   codes        6 x  4 KB  local TMA by the code warp (15) (full_c); freed by
-//                           the dequant warps once the codes are in
-//                           registers (empty_c)
+//   codes        6 x  4 KB  local TMA by the code warp (15) (full_c); a
+//                           dequant warp loads stage it + 3's codes into
+//                           registers right after decoding stage it, and
+//                           frees a stage's slot (empty_c) once its decode
+//                           has consumed them
 //   bf16 weight  6 x 16 KB  written by dequant group it % 3 after the MMA
 //                           freed the slot (empty_w); one arrive per warp
 //                           on the leader's full_w
@@ -91,7 +93,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint64_t* acc_full = empty_w + kPairRingW;                // local: accumulator complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile uint32_t* dep_scratch = reinterpret_cast<volatile uint32_t*>(bars + 64);   // one word per dequant thread
   auto par = [](int it, int depth) { return static_cast<uint32_t>((it / depth) & 1); };
   auto prev_par = [](int it, int depth) { return static_cast<uint32_t>(((it / depth) + 1) & 1); };
 
@@ -258,35 +259,32 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     load_raw(g, q0, s0);
     load_raw(g + G, q1, s1);
     load_raw(g + 2 * G, q2, s2);
-    for (int it = g; it < total; it += G) {
+    // codes of stage `it` into registers (after its full_c phase)
+    auto fetch = [&](int it, uint4& a0, uint4& a1) -> bool {
+      if (!mbar_wait(smem_u32(&full_c[it % kPairRingC]), par(it, kPairRingC), abort_flag, args.status)) return false;
+      const int64_t n = wn0 + wn_step * it, k = kb0 + kb_step * it;
+      if (it < args.num_kt && n < args.wN && k < KB) {
+        const uint8_t* cs = slot_c(it) + c_off;
+        a0 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 0) ^ c_swz) << 4));
+        a1 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 1) ^ c_swz) << 4));
+      } else {
+        a0 = make_uint4(0, 0, 0, 0); a1 = a0;
+      }
+      return true;
+    };
+    uint4 n0, n1;
+    bool live = g >= total || fetch(g, n0, n1);
+    for (int it = g; it < total && live; it += G) {
       const int ic = it % kPairRingC, iw = it % kPairRingW;
       const float scale = args.dq ? __fmul_rn(static_cast<float>(q0), s0) : s0;
-      if (!mbar_wait(smem_u32(&full_c[ic]), par(it, kPairRingC), abort_flag, args.status)) break;
+      const uint4 c0 = n0, c1 = n1;
       const int64_t n = wn0 + wn_step * it, k = kb0 + kb_step * it;
       const bool valid = it < args.num_kt && n < args.wN && k < KB;
-      uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-      if (valid) {
-        const uint8_t* cs = slot_c(it) + c_off;
-        c0 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 0) ^ c_swz) << 4));
-        c1 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 1) ^ c_swz) << 4));
-      }
-      // Release the codes slot only once the loads above have returned: an
-      // arrive does not wait for loads whose results are still unused, and
-      // the next TMA would overwrite the slot under them.  Storing a value
-      // computed from every loaded word makes the release wait for them.
-      dep_scratch[(warp - 2) * 32 + lane] = c0.x ^ c0.y ^ c0.z ^ c0.w ^ c1.x ^ c1.y ^ c1.z ^ c1.w;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&empty_c[ic]));   // codes are in registers: slot may refill
       // the bf16 slot is free once the MMA of its previous use has completed
       if (it >= kPairRingW &&
           !mbar_wait(smem_u32(&empty_w[iw]), prev_par(it, kPairRingW), abort_flag, args.status))
         break;
       if (it >= args.num_kt) {
-        // adapter stage: this CTA's adapter B half into the (now free) weight
-        // slot; its bytes complete on the leader's full_w of this stage,
-        // which this group has already seen advance past the slot's
-        // previous use (the empty_w wait above).  The expect comes before
-        // this warp's own arrive, so the phase cannot complete without it.
         if (((warp - 2) & 3) == 0 && lane == 0) {
           const int li = (it - args.num_kt) % nl1;
           const uint32_t fw = leader_bar(&full_w[iw]);
@@ -316,9 +314,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         fence_proxy_async_smem();
       }
+      // next own stage's codes: their loads run while this stage is handed over
+      if (it + G < total && !fetch(it + G, n0, n1)) live = false;
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_bar(&full_w[iw]));
-      // prefetch after the arrive, so that the arrive's release does not wait on these loads
+      if (lane == 0) {
+        mbar_arrive_cluster(leader_bar(&full_w[iw]));
+        mbar_arrive(smem_u32(&empty_c[ic]));   // this stage's codes were consumed by the stores above
+      }
       q0 = q1; s0 = s1; q1 = q2; s1 = s2;
       load_raw(it + 3 * G, q2, s2);
     }

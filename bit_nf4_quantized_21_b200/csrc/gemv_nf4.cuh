@@ -25,7 +25,9 @@
 //                column).  The weights never touch shared memory.
 //   warps 14..17 epilogue: accumulator (128 rows x 16 tokens, fp32) out of
 //                TMEM, plus the adapter term s T B^T in fp32, rounded once
-//                to bf16.
+//                to bf16.  Before its first tile these warps also compute
+//                the adapter's down-projection T = X A^T for the whole grid
+//                (below), while the other roles are already streaming.
 // MMA per slice: 8 x tcgen05.mma.cta_group::1.kind::f16, M 128 (weight
 // rows, A from TMEM), N 16 (tokens, B = activation slice, K-major, 128-byte
 // swizzle), K 16; each issuer's accumulator is double-buffered in TMEM so
@@ -44,7 +46,18 @@
 // the last of them to arrive: each writes its fp32 partial tile to the
 // workspace, bumps the tile's counter, and the CTA that sees the final count
 // adds the partials in CTA order (fixed order: deterministic), then applies
-// the epilogue.  No CTA ever waits for another.
+// the epilogue.  No CTA waits for another over a weight tile.
+//
+// Adapter down-projection T = X A^T [M, r] (fp32), folded into the same
+// launch: every CTA's epilogue threads (1) compute the partial of T over the
+// CTA's share of the contraction (K / G columns, CUDA cores, fp32, columns in
+// order) into partial slot c, (2) once every CTA has published its partial,
+// add up, in CTA order, the partials of the CTA's share of T's entries and
+// write them to T, and (3) once every CTA has done that, load s T into
+// shared memory for the epilogue.  The two grid-wide waits need every CTA
+// resident at once, which the launch guarantees (cooperative launch, one
+// CTA per SM); both are bounded like every other wait.  T is ready within a
+// few microseconds of the start, before the first tile's epilogue needs it.
 #pragma once
 #include "nf4_decode.cuh"
 
@@ -89,7 +102,11 @@ struct GvArgs {
   int M;                     // tokens (1..16)
   int r;                     // adapter rank
   float s;                   // alpha / r
-  const float* T;            // [M, r] fp32, X A^T (unscaled)
+  const __nv_bfloat16* X;    // [M, K] activations (row stride K)
+  const __nv_bfloat16* A;    // [r, K] adapter down-projection
+  float* T;                  // [M, r] fp32 out: X A^T (unscaled)
+  float* tpart;              // [G][M][r] partials of T
+  int* tcnt;                 // [2] grid arrival counters of the two T phases, zero on entry
   const __nv_bfloat16* B;    // [N, r]
   __nv_bfloat16* Y;          // [M, N]
   float* part;               // [kGvMaxCtas][2][128][16] partial tiles
@@ -158,6 +175,77 @@ __host__ __device__ __forceinline__ int64_t gv_cta_of(int64_t u, int64_t U, int6
 }
 __host__ __device__ __forceinline__ int64_t gv_begin(int64_t c, int64_t U, int64_t G) { return U * c / G; }
 
+// acc + sum over the 8 bf16 pairs of x and a, in element order (bf16 -> fp32
+// is exact: the 16 bits are the top half of the fp32 word)
+__device__ __forceinline__ float gv_dot8(uint4 x, uint4 a, float acc) {
+  const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, as[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc = fmaf(__uint_as_float(xs[i] << 16), __uint_as_float(as[i] << 16), acc);
+    acc = fmaf(__uint_as_float(xs[i] & 0xFFFF0000u), __uint_as_float(as[i] & 0xFFFF0000u), acc);
+  }
+  return acc;
+}
+
+// The 128 epilogue threads of this CTA publish their writes (fence, then one
+// arrival on the grid counter) and wait until all G CTAs have arrived.
+// Bounded: on timeout the CTA's abort flag and the timeout status are set.
+// Returns the same outcome in every one of the 128 threads.
+__device__ __forceinline__ bool gv_grid_arrive_wait(int* ctr, int64_t G, int et, volatile int* abort_flag,
+                                                    int* status) {
+  __threadfence();
+  named_bar_sync(1, 128);
+  bool ok = true;
+  if (et == 0) {
+    atomicAdd(ctr, 1);
+    const uint64_t t0 = global_ns();
+    while (true) {
+      int v;
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+      if (v >= G) break;
+      if (*abort_flag) { ok = false; break; }
+      if (global_ns() - t0 > QLORA_WAIT_NS) {
+        *abort_flag = 1;
+        if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
+        ok = false;
+        break;
+      }
+      __nanosleep(128);
+    }
+  }
+  ok = named_bar_and(1, 128, ok);
+  __threadfence();
+  return ok;
+}
+
+// T = X A^T for the whole grid, then s T into shared memory (see the header).
+__device__ __forceinline__ bool gv_adapter_T(const GvArgs& args, int64_t c, int64_t G, int et, float* sT,
+                                             volatile int* abort_flag) {
+  const int MR = args.M * args.r;
+  const int64_t K8 = args.K / 8;
+  const int64_t v0 = K8 * c / G, v1 = K8 * (c + 1) / G;
+  float* mine = args.tpart + c * MR;
+  for (int o = et; o < MR; o += 128) {
+    const int m = o / args.r, j = o - m * args.r;
+    const uint4* xp = reinterpret_cast<const uint4*>(args.X + static_cast<int64_t>(m) * args.K);
+    const uint4* ap = reinterpret_cast<const uint4*>(args.A + static_cast<int64_t>(j) * args.K);
+    float acc = 0.0f;
+    for (int64_t v = v0; v < v1; ++v) acc = gv_dot8(__ldg(xp + v), __ldg(ap + v), acc);
+    mine[o] = acc;
+  }
+  if (!gv_grid_arrive_wait(args.tcnt, G, et, abort_flag, args.status)) return false;
+  const int64_t o0 = MR * c / G, o1 = MR * (c + 1) / G;
+  for (int64_t o = o0 + et; o < o1; o += 128) {
+    float t = 0.0f;
+    for (int64_t cc = 0; cc < G; ++cc) t += __ldcg(args.tpart + cc * MR + o);
+    args.T[o] = t;
+  }
+  if (!gv_grid_arrive_wait(args.tcnt + 1, G, et, abort_flag, args.status)) return false;
+  for (int i = et; i < MR; i += 128) sT[i] = args.s * __ldcg(args.T + i);
+  named_bar_sync(1, 128);
+  return true;
+}
+
 __global__ void __launch_bounds__(kGvThreads, 1)
     k_gemv_nf4(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
                const GvArgs args) {
@@ -209,11 +297,6 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kGvTmemCols);
     tmem_relinquish();
-  }
-  if (warp >= kGvEpiWarp0) {
-    // s * T into shared memory (the adapter term of the epilogue)
-    const int n = args.M * args.r;
-    for (int i = threadIdx.x - kGvEpiWarp0 * 32; i < n; i += 128) sT[i] = args.s * args.T[i];
   }
   tc_fence_before();
   __syncthreads();
@@ -391,7 +474,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     const int64_t U = args.units;
     int64_t u = u0;
     int j = 0;
-    while (u < u1) {
+    const bool t_ok = gv_adapter_T(args, c, G, et, sT, abort_flag);
+    while (u < u1 && t_ok) {
       const int64_t t = u / KU;
       const int64_t seg_end = min(u1, (t + 1) * KU);
       const bool whole = (u == t * KU) && (seg_end == (t + 1) * KU);

@@ -211,7 +211,7 @@ qlora_status launch_skinny(const SkJob& j0, const SkJob* j1, cudaStream_t st) {
 
 // -------------------------------------------------------- workspace layout
 struct Ws {
-  size_t partial, partial2, cnt, t32, sx, ghl, thl, bpad, gv_part, gv_cnt, total;
+  size_t partial, partial2, cnt, t32, sx, ghl, thl, bpad, gv_part, gv_cnt, gv_tpart, total;
 };
 
 // Token counts up to this take the weight-streaming decode kernel.
@@ -252,6 +252,18 @@ SkPlans plans_of(const Dims& d) {
 // Arrival counters: T, G, dA, dB tiles, one 32-bit word each.
 size_t cnt_words(const SkPlans& p) { return p.T.ptiles + p.G.ptiles + p.dA.ptiles + p.dB.ptiles; }
 
+// The decode kernel's scratch (M <= 16): partial tiles, per-tile counters
+// followed by the two T-phase counters, and the partials of T.
+void gv_layout(const Dims& d, Ws& w, size_t& off) {
+  auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  w.gv_part = w.gv_cnt = w.gv_tpart = off;
+  if (d.M <= kDecodeMaxM) {
+    w.gv_part = off; off += a256(static_cast<size_t>(kGvMaxCtas) * 2 * kGvRows * kGvNT * 4);
+    w.gv_cnt = off; off += a256(static_cast<size_t>(cdiv(d.N, kGvRows) + 2) * 4);
+    w.gv_tpart = off; off += a256(static_cast<size_t>(kGvMaxCtas) * d.M * d.r * 4);
+  }
+}
+
 Ws ws_layout(const Dims& d) {
   const SkPlans pl = plans_of(d);
   auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
@@ -267,11 +279,7 @@ Ws ws_layout(const Dims& d) {
   w.ghl = off; off += a256(static_cast<size_t>(d.M) * d.Qh * 2);
   w.thl = off; off += a256(static_cast<size_t>(d.M) * d.Qh * 2);
   w.bpad = off; off += a256(static_cast<size_t>(d.N) * d.r8 * 2);
-  w.gv_part = w.gv_cnt = off;
-  if (d.M <= kDecodeMaxM) {
-    w.gv_part = off; off += a256(static_cast<size_t>(kGvMaxCtas) * 2 * kGvRows * kGvNT * 4);
-    w.gv_cnt = off; off += a256(static_cast<size_t>(cdiv(d.N, kGvRows)) * 4);
-  }
+  gv_layout(d, w, off);
   w.total = off;
   return w;
 }
@@ -415,11 +423,13 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   return QLORA_OK;
 }
 
-// Decode-shaped forward (M <= 16): Y = X W^T + s T B^T with T = X A^T in
-// fp32 at t32.  Persistent stream-K launch, one CTA per SM.
-qlora_status run_gemv(const void* X, const qlora_nf4_weight* Wq, const Dims& d, const float* t32, const void* B,
-                      void* Y, float alpha_over_r, uint8_t* ws, const Ws& L, const qlora_gemm_events* ev,
-                      int* status, cudaStream_t cs) {
+// Decode-shaped forward (M <= 16): Y = X W^T + s T B^T, with T = X A^T
+// computed in the same launch and written (fp32) to t32.  Persistent
+// stream-K launch, one CTA per SM, cooperative (every CTA resident at once:
+// the T phases wait across CTAs).  One memset clears the counters first.
+qlora_status run_gemv(const void* X, const void* A, const qlora_nf4_weight* Wq, const Dims& d, float* t32,
+                      const void* B, void* Y, float alpha_over_r, uint8_t* ws, const Ws& L,
+                      const qlora_gemm_events* ev, int* status, cudaStream_t cs) {
   if (d.r > kGvMaxRank) return QLORA_ERR_UNSUPPORTED;
   const int64_t tiles = cdiv(d.N, kGvRows);
   const int64_t KU = cdiv(d.K, kGvKS);
@@ -435,18 +445,32 @@ qlora_status run_gemv(const void* X, const qlora_nf4_weight* Wq, const Dims& d, 
   GvArgs a{};
   a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
   a.N = d.N; a.K = d.K; a.M = static_cast<int>(d.M); a.r = d.r; a.s = alpha_over_r;
+  a.X = static_cast<const __nv_bfloat16*>(X);
+  a.A = static_cast<const __nv_bfloat16*>(A);
   a.T = t32;
+  a.tpart = reinterpret_cast<float*>(ws + L.gv_tpart);
   a.B = static_cast<const __nv_bfloat16*>(B);
   a.Y = static_cast<__nv_bfloat16*>(Y);
   a.part = reinterpret_cast<float*>(ws + L.gv_part);
   a.cnt = reinterpret_cast<int*>(ws + L.gv_cnt);
+  a.tcnt = a.cnt + tiles;
   a.KU = KU;
   a.units = units;
   a.status = status;
-  if (cudaMemsetAsync(a.cnt, 0, static_cast<size_t>(tiles) * 4, cs) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaMemsetAsync(a.cnt, 0, static_cast<size_t>(tiles + 2) * 4, cs) != cudaSuccess) return QLORA_ERR_CUDA;
   if (ev && ev->gemm_start && cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_start), cs) != cudaSuccess)
     return QLORA_ERR_CUDA;
-  k_gemv_nf4<<<static_cast<unsigned>(grid), kGvThreads, kGvSmemBytes, cs>>>(tx, tc, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = kGvSmemBytes;
+  cfg.stream = cs;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_gemv_nf4, tx, tc, a) != cudaSuccess) return QLORA_ERR_CUDA;
   qlora_status rc = check_launch();
   if (rc == QLORA_OK && ev && ev->gemm_end &&
       cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_end), cs) != cudaSuccess)
@@ -547,14 +571,8 @@ qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* 
   float* t32 = T_save ? T_save : reinterpret_cast<float*>(ws + L.t32);
   __nv_bfloat16* sT = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
 
-  if (M <= kDecodeMaxM) {
-    // decode shape: T = X A^T (fp32), then the weight-streaming kernel
-    st = clear_counters(ws, L, plans_of(d), cs);
-    if (st != QLORA_OK) return st;
-    st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
-    if (st != QLORA_OK) return st;
-    return run_gemv(X, Wq, d, t32, B, Y, s, ws, L, events, d_status, cs);
-  }
+  if (M <= kDecodeMaxM)   // decode shape: one weight-streaming launch (T included)
+    return run_gemv(X, A, Wq, d, t32, B, Y, s, ws, L, events, d_status, cs);
 
   // 1. T = X A^T and s*T (bf16) for the fold
   st = clear_counters(ws, L, plans_of(d), cs);
@@ -690,11 +708,7 @@ Ws noalloc_fwd_layout(const Dims& d) {
   w.sx = off; off += a256(static_cast<size_t>(2 * d.M) * d.r8 * 2);
   w.ghl = w.thl = off;
   w.bpad = off; off += (d.r % 8) ? a256(static_cast<size_t>(d.N) * d.r8 * 2) : 0;
-  w.gv_part = w.gv_cnt = off;
-  if (d.M <= kDecodeMaxM) {
-    w.gv_part = off; off += a256(static_cast<size_t>(kGvMaxCtas) * 2 * kGvRows * kGvNT * 4);
-    w.gv_cnt = off; off += a256(static_cast<size_t>(cdiv(d.N, kGvRows)) * 4);
-  }
+  gv_layout(d, w, off);
   w.total = off;
   return w;
 }
@@ -724,13 +738,9 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const void* X, int64_t M, const
   float* t32 = T_save ? T_save : reinterpret_cast<float*>(ws + L.t32);
   __nv_bfloat16* sT = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
 
+  if (M <= kDecodeMaxM) return run_gemv(X, A, Wq, d, t32, B, Y, s, ws, L, nullptr, d_status, cs);
   st = clear_counters(ws, L, plans_of(d), cs);
   if (st != QLORA_OK) return st;
-  if (M <= kDecodeMaxM) {
-    st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
-    if (st != QLORA_OK) return st;
-    return run_gemv(X, Wq, d, t32, B, Y, s, ws, L, nullptr, d_status, cs);
-  }
 
   st = run_T(X, A, d, s, ws, L, t32, sT, d_status, cs);
   if (st != QLORA_OK) return st;

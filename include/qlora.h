@@ -153,12 +153,16 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  * T_save (nullable) fp32 [M, r]: T for the backward.  1 <= r <= 256.
  * M > 16: W^ is dequantised tile by tile in shared memory inside the
  * GEMM; the adapter product enters the same fp32 accumulator, one bf16
- * rounding per output.  M <= 16 (decode): a weight-streaming kernel
+ * rounding per output.  M <= 16 (decode): one weight-streaming launch
  * dequantises W^ straight into tensor memory, accumulates X W^T in fp32,
- * adds s T B^T in fp32 and rounds once; the workspace then also holds
- * per-CTA partial tiles and per-tile counters, which the call clears on
- * the stream before use.  Results are deterministic (fixed summation
- * order) for both paths.  Requires N % 8 == 0, K % 64 == 0.
+ * adds s T B^T in fp32 and rounds once; T = X A^T is computed in the same
+ * launch (fp32, CUDA cores) while the weights stream.  That launch is
+ * cooperative (one CTA per SM, all resident at once); if the device cannot
+ * co-schedule it (e.g. under a partition with fewer SMs than the device
+ * reports) the call returns QLORA_ERR_CUDA.  The workspace then also holds
+ * per-CTA partial tiles, partials of T and arrival counters, which the
+ * call clears on the stream before use.  Results are deterministic (fixed
+ * summation order) for both paths.  Requires N % 8 == 0, K % 64 == 0.
  */
 qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* Wq,
                               const void* A, const void* B, int r, float alpha,
@@ -201,8 +205,8 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M,
  * of s*T, a padded copy of B when r % 8 != 0) does not fit is rejected with
  * QLORA_ERR_SCRATCH_LIMIT before anything is enqueued; e.g. M = 8192,
  * r = 64 fits.  Every region is fully written before it is read, except
- * the decode path's (M <= 16) tile counters, which each call clears on
- * its stream before its kernels run.
+ * the arrival counters of the split-K and decode kernels, which each call
+ * clears on its stream before its kernels run.
  *
  * All calls on a device share the one array: calls whose work overlaps on
  * the GPU (different streams, or different host threads) race and give
