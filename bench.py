@@ -121,22 +121,35 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- our path
+# Input each projection reads: in a LLaMA decoder layer q, k and v project
+# the same normalised hidden state, and gate and up the same one.
+X_SOURCE = {"q": "q", "k": "q", "v": "q", "o": "o", "gate": "gate", "up": "gate", "down": "down"}
+
+
 class Layer:
-    """Seven NF4 projections of one layer, resident on the device."""
+    """Seven NF4 projections of one layer, resident on the device (q/k/v and
+    gate/up share their input tensor, as in the model)."""
 
     def __init__(self, q, wl, M, device, rank):
         self.q = q
         self.wl = wl
         self.M = M
         self.proj = []
+        index = {name: i for i, (name, _, _) in enumerate(wl.shapes)}
+        self.x = {}
         for i, (name, N, K) in enumerate(wl.shapes):
             seed = inputs.matrix_seed(wl.base_seed, rank, i)
+            xk = X_SOURCE[name]
+            if xk not in self.x:
+                self.x[xk] = inputs.normal((M, K), 1.0, inputs.matrix_seed(wl.base_seed, rank, index[xk]) * 16 + 1,
+                                           device)
             W = inputs.weight((N, K), wl.w_std, seed, device=device)
             Wq = q.empty_nf4(N, K, device)
             p = dict(name=name, N=N, K=K, W_bf16_bytes=W.numel() * 2)
             p["Wq"] = Wq
             p["W_tmp"] = W
-            p["X"] = inputs.normal((M, K), 1.0, seed * 16 + 1, device)
+            p["X"] = self.x[xk]
+            p["xkey"] = xk
             p["dY"] = inputs.normal((M, N), 1.0, seed * 16 + 2, device)
             p["A"] = inputs.normal((wl.r, K), 0.01, seed * 16 + 3, device)
             p["B"] = inputs.normal((N, wl.r), 0.01, seed * 16 + 4, device)
@@ -179,29 +192,33 @@ class Layer:
                                     d_status=self.status, gemm_events=ev)
 
     def step_e2e(self, hostX, hostdY, hostdA, hostdB, s_h2d, s_d2h, ev, allreduce=None):
-        """One step from pinned host buffers: each projection's inputs are
-        copied in on s_h2d while earlier projections compute (X in forward
-        order, then dY in backward order), each projection waits only for its
-        own inputs, and its gradients go back on s_d2h as soon as its backward
-        is done.  `ev` brackets the whole step on the compute stream."""
+        """One step from pinned host buffers: each distinct input X (hostX,
+        keyed like self.x) and each dY are copied in on s_h2d while earlier
+        projections compute (X in forward order of first use, then dY in
+        backward order), each projection waits only for its own inputs, and
+        its gradients go back on s_d2h as soon as its backward is done.
+        `ev` brackets the whole step on the compute stream."""
         q, alpha = self.q, self.wl.alpha
         comp = torch.cuda.current_stream()
         ev[0].record(comp)
         s_h2d.wait_event(ev[0])
-        ready_x, ready_dy = [], {}
+        ready_x, ready_dy = {}, {}
         with torch.cuda.stream(s_h2d):
-            for p, hx in zip(self.proj, hostX):
-                p["X"].copy_(hx, non_blocking=True)
+            for p in self.proj:
+                xk = p["xkey"]
+                if xk in ready_x:
+                    continue
+                self.x[xk].copy_(hostX[xk], non_blocking=True)
                 e = torch.cuda.Event()
                 e.record(s_h2d)
-                ready_x.append(e)
+                ready_x[xk] = e
             for i in reversed(range(len(self.proj))):
                 self.proj[i]["dY"].copy_(hostdY[i], non_blocking=True)
                 e = torch.cuda.Event()
                 e.record(s_h2d)
                 ready_dy[i] = e
-        for p, e in zip(self.proj, ready_x):
-            comp.wait_event(e)
+        for p in self.proj:
+            comp.wait_event(ready_x[p["xkey"]])
             q.qlora_linear_fwd(p["X"], p["Wq"], p["A"], p["B"], alpha, Y=p["Y"], T_save=p["T"],
                                workspace=self.ws, d_status=self.status)
         done = {}
@@ -349,11 +366,11 @@ def run_ours(args):
     # ---- end to end through host buffers (pinned), copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        hostX = [p["X"].cpu().pin_memory() for p in layer.proj]
+        hostX = {k: x.cpu().pin_memory() for k, x in layer.x.items()}
         hostdY = [p["dY"].cpu().pin_memory() for p in layer.proj]
         hostdA = [torch.empty_like(p["dA"], device="cpu").pin_memory() for p in layer.proj]
         hostdB = [torch.empty_like(p["dB"], device="cpu").pin_memory() for p in layer.proj]
-        h2d = sum(t.numel() * t.element_size() for t in hostX + hostdY)
+        h2d = sum(t.numel() * t.element_size() for t in list(hostX.values()) + hostdY)
         d2h = sum(t.numel() * t.element_size() for t in hostdA + hostdB)
         e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(args.steps)]
@@ -400,6 +417,7 @@ def run_ours(args):
         "config": {"workload": "llama7b-layer-7proj-fwd+bwd", "tokens_per_gpu": WL.M,
                    "batch": 4, "seq_len": 512, "lora_r": WL.r, "lora_alpha": WL.alpha,
                    "projections": [[n, N, K] for n, N, K in WL.shapes],
+                   "inputs": "q/k/v read one X, gate/up another (as in the decoder layer)",
                    "weights": "NF4 double-quant, block 64, group 256",
                    "flops_per_step": step_flops(), "l2": "flushed between timed steps",
                    "parallelism": f"dp{world}"},
@@ -467,11 +485,11 @@ def _quantize_model(q, wl, dev, status):
 def _layer_tensors(wl, L, M, dev, x_shared=True):
     """Adapters and activations of one layer.  With x_shared, q/k/v read one
     input and gate/up another, as in a LLaMA decoder layer."""
-    xkey = {0: 0, 1: 0, 2: 0, 3: 3, 4: 4, 5: 4, 6: 6} if x_shared else {i: i for i in range(7)}
+    index = {name: i for i, (name, _, _) in enumerate(wl.shapes)}
     xs, out = {}, []
     for i, (name, N, K) in enumerate(wl.shapes):
         seed = inputs.matrix_seed(wl.base_seed, L, i)
-        k = xkey[i]
+        k = index[X_SOURCE[name]] if x_shared else i
         if k not in xs:
             xs[k] = inputs.normal((M, K), 1.0, inputs.matrix_seed(wl.base_seed, L, k) * 16 + 1, dev)
         out.append(dict(X=xs[k], dY=inputs.normal((M, N), 1.0, seed * 16 + 2, dev),
