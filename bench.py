@@ -121,6 +121,41 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- our path
+def grad_buffer(shapes, r, device):
+    """One flat fp32 buffer holding every projection's dA [r, K] and dB [N, r]
+    as consecutive views: the kernels write the gradients straight into it and
+    the data-parallel sum is one in-place all-reduce.  Returns (flat, [(dA, dB)
+    per projection]).  Every view starts on a 16-byte boundary (K % 64 == 0,
+    N % 8 == 0)."""
+    sizes = []
+    for _, N, K in shapes:
+        sizes += [(r, K), (N, r)]
+    flat = torch.zeros(sum(a * b for a, b in sizes), dtype=torch.float32, device=device)
+    views, off = [], 0
+    for a, b in sizes:
+        views.append(flat[off:off + a * b].view(a, b))
+        off += a * b
+    return flat, [(views[2 * i], views[2 * i + 1]) for i in range(len(shapes))]
+
+
+def allreduce_sum(flat, world):
+    """Data parallel: every rank ends with the sum of the gradients over all
+    ranks (the step's loss is the sum over every rank's tokens)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(flat)
+
+
+def max_over_ranks(x, world, device):
+    """Slowest rank's value of a per-rank time."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # Input each projection reads: in a LLaMA decoder layer q, k and v project
 # the same normalised hidden state, and gate and up the same one.
 X_SOURCE = {"q": "q", "k": "q", "v": "q", "o": "o", "gate": "gate", "up": "gate", "down": "down"}
@@ -135,6 +170,7 @@ class Layer:
         self.wl = wl
         self.M = M
         self.proj = []
+        self.grad_flat, grads = grad_buffer(wl.shapes, wl.r, device)
         index = {name: i for i, (name, _, _) in enumerate(wl.shapes)}
         self.x = {}
         for i, (name, N, K) in enumerate(wl.shapes):
@@ -156,14 +192,11 @@ class Layer:
             p["Y"] = torch.empty((M, N), dtype=torch.bfloat16, device=device)
             p["T"] = torch.empty((M, wl.r), dtype=torch.float32, device=device)
             p["dX"] = torch.empty((M, K), dtype=torch.bfloat16, device=device)
-            p["dA"] = torch.empty((wl.r, K), dtype=torch.float32, device=device)
-            p["dB"] = torch.empty((N, wl.r), dtype=torch.float32, device=device)
+            p["dA"], p["dB"] = grads[i]
             self.proj.append(p)
         ws = max(q.qlora_workspace_bytes(M, p["N"], p["K"], wl.r) for p in self.proj)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
-        # flat gradient buffer for the data-parallel all-reduce
-        self.grad_numel = sum(p["dA"].numel() + p["dB"].numel() for p in self.proj)
 
     def quantize_all(self, events=None):
         for p in self.proj:
@@ -305,17 +338,9 @@ def run_ours(args):
     assert layer.status.item() == 0, "quantiser reported non-finite weights"
 
     l2buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    grad_flat = torch.empty(layer.grad_numel, dtype=torch.float32, device=dev)
 
     def allreduce_grads():
-        if world == 1:
-            return
-        off = 0
-        for p in layer.proj:
-            for t in (p["dA"], p["dB"]):
-                grad_flat[off:off + t.numel()].copy_(t.view(-1))
-                off += t.numel()
-        dist.all_reduce(grad_flat)
+        allreduce_sum(layer.grad_flat, world)
 
     # ---- warm-up
     for _ in range(args.warmup):
@@ -345,11 +370,7 @@ def run_ours(args):
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     gemm_ms = [[a.elapsed_time(b) for a, b in evs] for evs in gemm_ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     assert layer.status.item() == 0, f"device status {layer.status.item()}"
     flops = step_flops() * args.steps * world
     value = flops / (total_ms * 1e-3) / 1e12
@@ -382,11 +403,7 @@ def run_ours(args):
             layer.step_e2e(hostX, hostdY, hostdA, hostdB, s_h2d, s_d2h, e_ev[i], allreduce_grads if world > 1 else None)
         torch.cuda.synchronize()
         barrier()
-        e_ms = sum(a.elapsed_time(b) for a, b in e_ev)
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), world, dev)
         e2e = {"value": round(flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e_ms / args.steps, 4)}
