@@ -224,6 +224,18 @@ class Layer:
                                     dX=p["dX"], dA=p["dA"], dB=p["dB"], workspace=self.ws,
                                     d_status=self.status, gemm_events=ev)
 
+    def step_dense(self, Wd):
+        """The same step over dense bf16 weights Wd (one per projection):
+        plain LoRA through the same GEMM, the baseline QLoRA is compared to."""
+        alpha = self.wl.alpha
+        for p, W in zip(self.proj, Wd):
+            self.q.qlora_lora_linear_fwd(p["X"], W, p["A"], p["B"], alpha, Y=p["Y"], T_save=p["T"],
+                                         workspace=self.ws, d_status=self.status)
+        for p, W in zip(reversed(self.proj), reversed(Wd)):
+            self.q.qlora_lora_linear_bwd(p["dY"], p["X"], W, p["A"], p["B"], alpha, T_saved=p["T"],
+                                         dX=p["dX"], dA=p["dA"], dB=p["dB"], workspace=self.ws,
+                                         d_status=self.status)
+
     def step_e2e(self, hostX, hostdY, hostdA, hostdB, s_h2d, s_d2h, ev, allreduce=None):
         """One step from pinned host buffers: each distinct input X (hostX,
         keyed like self.x) and each dY are copied in on s_h2d while earlier
@@ -610,6 +622,21 @@ def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_param
     out["dequantize"] = {"value": round(dgbs, 1), "unit": "GB/s", "shape": [p["N"], p["K"]],
                          "frac_of_hbm": round(dgbs / hbm, 4)}
     del Wout
+    # plain LoRA on a bf16 base (the weights' dequantised copies) through the
+    # same GEMM, timed with the same harness as the NF4 step beside it: the
+    # pages say QLoRA steps are slower than LoRA's without giving a number
+    Wd = [q.qlora_dequantize(p["Wq"]) for p in layer.proj]
+    for _ in range(3):
+        layer.step_dense(Wd)
+    ms_d = statistics.median(time_events(lambda: layer.step_dense(Wd), 10, flush=lambda: l2buf.add_(1)))
+    ms_q = statistics.median(time_events(layer.step, 10, flush=lambda: l2buf.add_(1)))
+    assert layer.status.item() == 0, f"device status {layer.status.item()}"
+    out["lora_bf16_baseline"] = {"value": round(step_flops() / (ms_d * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                                 "ms_per_step": round(ms_d, 4), "qlora_ms_per_step": round(ms_q, 4),
+                                 "qlora_over_lora_time": round(ms_q / ms_d, 4),
+                                 "weights": "bf16 copies of the layer's NF4 weights (dequantised)"}
+    del Wd
+    torch.cuda.empty_cache()
     # decode-shaped forward: 70B MLP weights, M in {1, 4, 16}
     wl = inputs.DECODE
     dec = {}

@@ -37,6 +37,12 @@
 // slots because each ring depth is a multiple of its waiters' G, so no
 // waiter can be two phases behind and the 1-bit phase parity is safe.
 // Epilogue: every CTA reads its own TMEM half (tcgen05.ld) and writes bf16.
+//
+// WDENSE = true is the same GEMM over a dense bf16 weight (plain LoRA, the
+// baseline the QLoRA pages compare against): the weight tile of every
+// stage arrives by TMA straight into the weight slot, the way the adapter
+// stages' B tiles do (tm_codes then maps the bf16 weight), and nothing is
+// dequantised.
 #pragma once
 #include "nf4_decode.cuh"
 #include "gemm_nf4.cuh"
@@ -73,7 +79,7 @@ constexpr uint32_t kPairSmemBytes = kPairOffBar + 1024 /*align*/ + 512 /*bars*/ 
 constexpr uint32_t kPairTmemCols = 512;   // D0 (even stages) at 0, D1 (odd stages) at 256
 static_assert(kPairSmemBytes <= 227 * 1024, "pair kernel shared memory");
 
-template <int MODE>
+template <int MODE, bool WDENSE = false>
 __global__ void __launch_bounds__(kPairThreads, 1)
     k_gemm_nf4_pair(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                     const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
@@ -182,14 +188,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             !mbar_wait(smem_u32(&empty_c[ic]), prev_par(it, kPairRingC), abort_flag, args.status))
           break;
         const uint32_t fc = smem_u32(&full_c[ic]);
-        if (it < args.num_kt) {
+        if (it < args.num_kt && !WDENSE) {
           mbar_arrive_expect_tx(fc, kPairCBytes);
           if (MODE == kModeFwd)
             tma_load_2d(smem_u32(slot_c(it)), &tm_codes, fc, it * 32, static_cast<int32_t>(nc0));
           else
             tma_load_2d(smem_u32(slot_c(it)), &tm_codes, fc, static_cast<int32_t>(nc0 / 2), it * 64);
         } else {
-          mbar_arrive(fc);   // no codes in adapter stages: keeps the dequant warps' phases in step
+          mbar_arrive(fc);   // no codes (adapter stage, dense weight): keeps the dequant warps' phases in step
         }
         ++issued;
       }
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     // raw block-scale inputs of this thread's stages, loaded 3 own stages ahead
     auto load_raw = [&](int it, uint32_t& rq, float& rs) {
       rq = 0; rs = 0.0f;
-      if (it >= args.num_kt) return;
+      if (it >= args.num_kt || WDENSE) return;
       const int64_t n = wn0 + wn_step * it, k = kb0 + kb_step * it;
       if (n >= args.wN || k >= KB) return;
       const int64_t f = n * KB + k;
@@ -263,7 +269,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     auto fetch = [&](int it, uint4& a0, uint4& a1) -> bool {
       if (!mbar_wait(smem_u32(&full_c[it % kPairRingC]), par(it, kPairRingC), abort_flag, args.status)) return false;
       const int64_t n = wn0 + wn_step * it, k = kb0 + kb_step * it;
-      if (it < args.num_kt && n < args.wN && k < KB) {
+      if (it < args.num_kt && n < args.wN && k < KB && !WDENSE) {
         const uint8_t* cs = slot_c(it) + c_off;
         a0 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 0) ^ c_swz) << 4));
         a1 = *reinterpret_cast<const uint4*>(cs + (((c_ch0 + 1) ^ c_swz) << 4));
@@ -284,16 +290,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       if (it >= kPairRingW &&
           !mbar_wait(smem_u32(&empty_w[iw]), prev_par(it, kPairRingW), abort_flag, args.status))
         break;
-      if (it >= args.num_kt) {
+      if (it >= args.num_kt || WDENSE) {
+        // the stage's B operand by TMA: the adapter tile, or the dense weight
+        // tile (rows/columns past the weight's edge arrive as zeros)
         if (((warp - 2) & 3) == 0 && lane == 0) {
-          const int li = (it - args.num_kt) % nl1;
+          const bool lora = it >= args.num_kt;
+          const CUtensorMap* map = lora ? &tm_lb : &tm_codes;
+          const int32_t kk = lora ? ((it - args.num_kt) % nl1) * 64 : it * 64;
           const uint32_t fw = leader_bar(&full_w[iw]);
           mbar_expect_tx_cluster(fw, kPairWBytes);
           if (MODE == kModeFwd) {
-            tma_load_2d_pair(smem_u32(slot_w(it)), &tm_lb, fw, li * 64, static_cast<int32_t>(nc0));
+            tma_load_2d_pair(smem_u32(slot_w(it)), map, fw, kk, static_cast<int32_t>(nc0));
           } else {
-            tma_load_2d_pair(smem_u32(slot_w(it)), &tm_lb, fw, static_cast<int32_t>(nc0), li * 64);
-            tma_load_2d_pair(smem_u32(slot_w(it)) + 8192, &tm_lb, fw, static_cast<int32_t>(nc0) + 64, li * 64);
+            tma_load_2d_pair(smem_u32(slot_w(it)), map, fw, static_cast<int32_t>(nc0), kk);
+            tma_load_2d_pair(smem_u32(slot_w(it)) + 8192, map, fw, static_cast<int32_t>(nc0) + 64, kk);
           }
         }
       } else {
@@ -328,7 +338,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     // flight into shared memory, and nobody else waits for them: give them
     // time to land before the CTA can exit (error path only; a tile load
     // takes microseconds).
-    if (*abort_flag && ((warp - 2) & 3) == 0 && lane == 0 && total > args.num_kt) {
+    if (*abort_flag && ((warp - 2) & 3) == 0 && lane == 0 && (WDENSE || total > args.num_kt)) {
       const uint64_t t0 = global_ns();
       while (global_ns() - t0 < 1000000ull) {}
     }

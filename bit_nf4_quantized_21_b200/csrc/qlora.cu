@@ -86,6 +86,8 @@ bool ensure_smem_attrs() {
   ok = ok && cudaFuncSetAttribute(k_gemm_nf4<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeFwd>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeFwd, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeDx, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
@@ -361,20 +363,30 @@ qlora_status launch_gemm(int mode, const CUtensorMap& tact, const CUtensorMap& t
 // 2-SM pair kernel (256 x 256 tiles per pair), smaller M the 1-CTA kernel.
 //   fwd: act = X [M, K], la = s*T planes [2M, r8], lb = B [N, r8], out Y [M, N]
 //   dX : act = dY [M, N], la = s*G planes [2M, r8], lb = A [r, K], out dX [M, K]
-qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, const Dims& d, const void* la,
-                       const void* lb, void* out, const qlora_gemm_events* ev, int* status, cudaStream_t cs) {
-  const bool pair = d.M > 128;
+// The fused GEMM of the forward (mode kModeFwd) or of dX (kModeDx), over
+// the NF4 weight Wq or, when Wdense is given, over a dense bf16 weight
+// [N, K] (plain LoRA; always the 2-SM pair kernel).
+qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, const void* Wdense, const Dims& d,
+                       const void* la, const void* lb, void* out, const qlora_gemm_events* ev, int* status,
+                       cudaStream_t cs) {
+  const bool dense = Wdense != nullptr;
+  const bool pair = d.M > 128 || dense;
   const bool fwd = mode == kModeFwd;
   CUtensorMap tact, tcodes, tla, tlb;
   if (fwd) {
     if (!bf16_map(&tact, act, d.K, d.M, d.K, 64, 128)) return QLORA_ERR_CUDA;
-    if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 32, pair ? 128 : kGemmBN,
-                  CU_TENSOR_MAP_SWIZZLE_32B))
+    if (dense) {
+      if (!bf16_map(&tcodes, Wdense, d.K, d.N, d.K, 64, 128)) return QLORA_ERR_CUDA;
+    } else if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 32,
+                         pair ? 128 : kGemmBN, CU_TENSOR_MAP_SWIZZLE_32B)) {
       return QLORA_ERR_CUDA;
+    }
     if (!bf16_map(&tlb, lb, d.r8, d.N, d.r8, 64, pair ? 128 : kGemmBN)) return QLORA_ERR_CUDA;
   } else {
     if (!bf16_map(&tact, act, d.N, d.M, d.N, 64, 128)) return QLORA_ERR_CUDA;
-    if (pair) {
+    if (dense) {
+      if (!bf16_map(&tcodes, Wdense, d.K, d.N, d.K, 64, 64)) return QLORA_ERR_CUDA;
+    } else if (pair) {
       if (!make_map(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq->codes, d.K / 2, d.N, d.K / 2, 64, 64,
                     CU_TENSOR_MAP_SWIZZLE_64B))
         return QLORA_ERR_CUDA;
@@ -387,7 +399,9 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   }
   if (!bf16_map(&tla, la, d.r8, 2 * d.M, d.r8, 64, 128)) return QLORA_ERR_CUDA;
   GemmArgs a{};
-  a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
+  if (!dense) {
+    a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
+  }
   a.wN = d.N; a.wK = d.K; a.M = d.M;
   a.out_cols = fwd ? d.N : d.K;
   a.ldo = a.out_cols;
@@ -412,8 +426,13 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd>, tact, tcodes, tla, tlb, a)
-                      : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx>, tact, tcodes, tla, tlb, a);
+  cudaError_t e;
+  if (dense)
+    e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, true>, tact, tcodes, tla, tlb, a)
+            : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, true>, tact, tcodes, tla, tlb, a);
+  else
+    e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd>, tact, tcodes, tla, tlb, a)
+            : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx>, tact, tcodes, tla, tlb, a);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return QLORA_ERR_CUDA;
@@ -476,6 +495,96 @@ qlora_status run_gemv(const void* X, const void* A, const qlora_nf4_weight* Wq, 
       cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_end), cs) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return rc;
+}
+
+// Backward body shared by the NF4 entry (Wq) and the dense-bf16 one (Wdense):
+// arguments already validated.
+qlora_status linear_bwd_core(const void* dY, const void* X, const Dims& d, const qlora_nf4_weight* Wq,
+                             const void* Wdense, const void* A, const void* B, float alpha, const float* T_saved,
+                             void* dX, void* dA, void* dB, qlora_dtype grad_dtype, void* workspace, int* d_status,
+                             const qlora_gemm_events* events, cudaStream_t cs) {
+  qlora_status st = QLORA_OK;
+  const Ws L = ws_layout(d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const float s = alpha / static_cast<float>(d.r);
+  const SkPlans P = plans_of(d);
+  __nv_bfloat16* sG = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
+  __nv_bfloat16* Ghl = reinterpret_cast<__nv_bfloat16*>(ws + L.ghl);
+  __nv_bfloat16* Thl = reinterpret_cast<__nv_bfloat16*>(ws + L.thl);
+
+  const void* Bp = padded_B(B, d, ws, L, cs, &st);
+  if (st != QLORA_OK) return st;
+  st = clear_counters(ws, L, P, cs);
+  if (st != QLORA_OK) return st;
+  // 0. T recomputed when the forward's was not kept
+  const float* t = T_saved;
+  if (!t) {
+    float* t32 = reinterpret_cast<float*>(ws + L.t32);
+    st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
+    if (st != QLORA_OK) return st;
+    t = t32;
+  }
+  // 1. G = dY B -> s*G (bf16 planes, for the dX fold) and [G_hi | G_lo] (for
+  //    dA); the same launch turns T into [T_hi | T_lo] (for dB)
+  {
+    SkJob j;
+    j.pl = P.G;
+    if (!bf16_map(&j.ta, dY, d.N, d.M, d.N, 64, kSkBM)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&j.tb, Bp, d.r8, d.N, d.r8, 64, 64)) return QLORA_ERR_CUDA;
+    j.a = sk_args(j.pl, reinterpret_cast<float*>(ws + L.partial), cnt_G(ws, L, P), d_status);
+    sk_rows(j.a, d, s, nullptr, sG, Ghl);
+    j.a.side_src = t;
+    j.a.side_rows = d.M;
+    j.a.side_hl = Thl;
+    st = launch_skinny<0, 1>(j, nullptr, cs);
+    if (st != QLORA_OK) return st;
+  }
+  // 2. dX = dY W^ + (sG) A
+  if (dX) {
+    st = run_fused(kModeDx, dY, Wq, Wdense, d, sG, A, dX, events, d_status, cs);
+    if (st != QLORA_OK) return st;
+  }
+  // 3. dA = s G^T X (C[k, q] = sum_m X[m, k] Ghl[m, q]) and dB = s dY^T T
+  //    (C[n, q] = sum_m dY[m, n] Thl[m, q]) in one launch
+  {
+    const int out_bf16 = grad_dtype == QLORA_BF16 ? 1 : 0;
+    SkJob ja, jb;
+    ja.pl = P.dA;
+    jb.pl = P.dB;
+    if (!bf16_map(&ja.ta, X, d.K, d.M, d.K, 64, 64)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&ja.tb, Ghl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&jb.ta, dY, d.N, d.M, d.N, 64, 64)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&jb.tb, Thl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
+    ja.a = sk_args(ja.pl, reinterpret_cast<float*>(ws + L.partial), cnt_dA(ws, L, P), d_status);
+    jb.a = sk_args(jb.pl, reinterpret_cast<float*>(ws + L.partial2), cnt_dB(ws, L, P), d_status);
+    for (SkinnyArgs* a : {&ja.a, &jb.a}) {
+      a->finish = kFinGrad;
+      a->s = s; a->r = d.r; a->r8 = d.r8; a->r16 = d.r16; a->Qh = d.Qh;
+      a->out_bf16 = out_bf16;
+    }
+    ja.a.transpose = 1;
+    ja.a.out = dA;
+    jb.a.transpose = 0;
+    jb.a.out = dB;
+    st = launch_skinny<1, 1>(ja, &jb, cs);
+  }
+  return st;
+}
+
+// Validation of the dense-bf16 entries: the same shape rules as the NF4
+// weight (N % 8 == 0, K % 64 == 0, 1 <= r <= 256).
+qlora_status check_dense(int64_t M, const void* W, int64_t N, int64_t K, int r, float alpha, const void* workspace,
+                         size_t ws_bytes) {
+  if (!W || !aligned16(W)) return QLORA_ERR_INVALID_ARG;
+  if (N < 1 || K < 64 || (K % 64) != 0) return QLORA_ERR_INVALID_ARG;
+  if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
+  if (N % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (M < 1 || M > (int64_t(1) << 31)) return QLORA_ERR_INVALID_ARG;
+  if (r < 1 || r > 256) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  if (ws_bytes < ws_layout(dims_of(M, N, K, r)).total) return QLORA_ERR_WORKSPACE;
+  return QLORA_OK;
 }
 
 }  // namespace
@@ -583,7 +692,7 @@ qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* 
   if (st != QLORA_OK) return st;
 
   // 2. Y = X W^T + (sT) B^T
-  return run_fused(kModeFwd, X, Wq, d, sT, Bp, Y, events, d_status, cs);
+  return run_fused(kModeFwd, X, Wq, nullptr, d, sT, Bp, Y, events, d_status, cs);
 }
 
 qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const qlora_nf4_weight* Wq, const void* A,
@@ -600,71 +709,49 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
   if (!ensure_smem_attrs()) return QLORA_ERR_CUDA;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const Dims d = dims_of(M, Wq->rows, Wq->cols, r);
+  return linear_bwd_core(dY, X, d, Wq, nullptr, A, B, alpha, T_saved, dX, dA, dB, grad_dtype, workspace, d_status,
+                         events, cs);
+}
+
+qlora_status qlora_lora_linear_fwd(const void* X, int64_t M, const void* W, int64_t N, int64_t K, const void* A,
+                                   const void* B, int r, float alpha, void* Y, float* T_save, void* workspace,
+                                   size_t ws_bytes, int* d_status, const qlora_gemm_events* events, void* stream) {
+  qlora_status st = check_dense(M, W, N, K, r, alpha, workspace, ws_bytes);
+  if (st != QLORA_OK) return st;
+  if (!X || !A || !B || !Y || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y))
+    return QLORA_ERR_INVALID_ARG;
+  if (T_save && !aligned16(T_save)) return QLORA_ERR_INVALID_ARG;
+  if (!ensure_smem_attrs()) return QLORA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const Dims d = dims_of(M, N, K, r);
   const Ws L = ws_layout(d);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const float s = alpha / static_cast<float>(r);
-  const SkPlans P = plans_of(d);
-  __nv_bfloat16* sG = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
-  __nv_bfloat16* Ghl = reinterpret_cast<__nv_bfloat16*>(ws + L.ghl);
-  __nv_bfloat16* Thl = reinterpret_cast<__nv_bfloat16*>(ws + L.thl);
-
+  float* t32 = T_save ? T_save : reinterpret_cast<float*>(ws + L.t32);
+  __nv_bfloat16* sT = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
+  st = clear_counters(ws, L, plans_of(d), cs);
+  if (st != QLORA_OK) return st;
+  st = run_T(X, A, d, s, ws, L, t32, sT, d_status, cs);
+  if (st != QLORA_OK) return st;
   const void* Bp = padded_B(B, d, ws, L, cs, &st);
   if (st != QLORA_OK) return st;
-  st = clear_counters(ws, L, P, cs);
+  return run_fused(kModeFwd, X, nullptr, W, d, sT, Bp, Y, events, d_status, cs);
+}
+
+qlora_status qlora_lora_linear_bwd(const void* dY, const void* X, int64_t M, const void* W, int64_t N, int64_t K,
+                                   const void* A, const void* B, int r, float alpha, const float* T_saved, void* dX,
+                                   void* dA, void* dB, qlora_dtype grad_dtype, void* workspace, size_t ws_bytes,
+                                   int* d_status, const qlora_gemm_events* events, void* stream) {
+  qlora_status st = check_dense(M, W, N, K, r, alpha, workspace, ws_bytes);
   if (st != QLORA_OK) return st;
-  // 0. T recomputed when the forward's was not kept
-  const float* t = T_saved;
-  if (!t) {
-    float* t32 = reinterpret_cast<float*>(ws + L.t32);
-    st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
-    if (st != QLORA_OK) return st;
-    t = t32;
-  }
-  // 1. G = dY B -> s*G (bf16 planes, for the dX fold) and [G_hi | G_lo] (for
-  //    dA); the same launch turns T into [T_hi | T_lo] (for dB)
-  {
-    SkJob j;
-    j.pl = P.G;
-    if (!bf16_map(&j.ta, dY, d.N, d.M, d.N, 64, kSkBM)) return QLORA_ERR_CUDA;
-    if (!bf16_map(&j.tb, Bp, d.r8, d.N, d.r8, 64, 64)) return QLORA_ERR_CUDA;
-    j.a = sk_args(j.pl, reinterpret_cast<float*>(ws + L.partial), cnt_G(ws, L, P), d_status);
-    sk_rows(j.a, d, s, nullptr, sG, Ghl);
-    j.a.side_src = t;
-    j.a.side_rows = d.M;
-    j.a.side_hl = Thl;
-    st = launch_skinny<0, 1>(j, nullptr, cs);
-    if (st != QLORA_OK) return st;
-  }
-  // 2. dX = dY W^ + (sG) A
-  if (dX) {
-    st = run_fused(kModeDx, dY, Wq, d, sG, A, dX, events, d_status, cs);
-    if (st != QLORA_OK) return st;
-  }
-  // 3. dA = s G^T X (C[k, q] = sum_m X[m, k] Ghl[m, q]) and dB = s dY^T T
-  //    (C[n, q] = sum_m dY[m, n] Thl[m, q]) in one launch
-  {
-    const int out_bf16 = grad_dtype == QLORA_BF16 ? 1 : 0;
-    SkJob ja, jb;
-    ja.pl = P.dA;
-    jb.pl = P.dB;
-    if (!bf16_map(&ja.ta, X, d.K, d.M, d.K, 64, 64)) return QLORA_ERR_CUDA;
-    if (!bf16_map(&ja.tb, Ghl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
-    if (!bf16_map(&jb.ta, dY, d.N, d.M, d.N, 64, 64)) return QLORA_ERR_CUDA;
-    if (!bf16_map(&jb.tb, Thl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
-    ja.a = sk_args(ja.pl, reinterpret_cast<float*>(ws + L.partial), cnt_dA(ws, L, P), d_status);
-    jb.a = sk_args(jb.pl, reinterpret_cast<float*>(ws + L.partial2), cnt_dB(ws, L, P), d_status);
-    for (SkinnyArgs* a : {&ja.a, &jb.a}) {
-      a->finish = kFinGrad;
-      a->s = s; a->r = d.r; a->r8 = d.r8; a->r16 = d.r16; a->Qh = d.Qh;
-      a->out_bf16 = out_bf16;
-    }
-    ja.a.transpose = 1;
-    ja.a.out = dA;
-    jb.a.transpose = 0;
-    jb.a.out = dB;
-    st = launch_skinny<1, 1>(ja, &jb, cs);
-  }
-  return st;
+  if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(dA) || !aligned16(dB))
+    return QLORA_ERR_INVALID_ARG;
+  if ((dX && !aligned16(dX)) || (T_saved && !aligned16(T_saved))) return QLORA_ERR_INVALID_ARG;
+  if (grad_dtype != QLORA_F32 && grad_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (!ensure_smem_attrs()) return QLORA_ERR_CUDA;
+  return linear_bwd_core(dY, X, dims_of(M, N, K, r), nullptr, W, A, B, alpha, T_saved, dX, dA, dB, grad_dtype,
+                         workspace, d_status, events, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -747,5 +834,5 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const void* X, int64_t M, const
   const void* Bp = padded_B(B, d, ws, L, cs, &st);
   if (st != QLORA_OK) return st;
 
-  return run_fused(kModeFwd, X, Wq, d, sT, Bp, Y, nullptr, d_status, cs);
+  return run_fused(kModeFwd, X, Wq, nullptr, d, sT, Bp, Y, nullptr, d_status, cs);
 }

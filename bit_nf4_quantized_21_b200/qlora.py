@@ -27,7 +27,7 @@ DEV_TIMEOUT = 2
 EXPORTED = (
     "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
-    "qlora_version", "qlora_linear_fwd_noalloc",
+    "qlora_version", "qlora_linear_fwd_noalloc", "qlora_lora_linear_fwd", "qlora_lora_linear_bwd",
 )
 
 
@@ -95,6 +95,12 @@ def lib() -> ctypes.CDLL:
             L.qlora_linear_fwd_noalloc.argtypes = [P, I64, ctypes.POINTER(NF4WeightC), P, P, I32, F, P,
                                                    P, P, P]
             L.qlora_linear_fwd_noalloc.restype = I32
+            L.qlora_lora_linear_fwd.argtypes = [P, I64, P, I64, I64, P, P, I32, F, P, P, P, ctypes.c_size_t,
+                                                P, P, P]
+            L.qlora_lora_linear_fwd.restype = I32
+            L.qlora_lora_linear_bwd.argtypes = [P, P, I64, P, I64, I64, P, P, I32, F, P, P, P, P, I32, P,
+                                                ctypes.c_size_t, P, P, P]
+            L.qlora_lora_linear_bwd.restype = I32
             L.qlora_status_string.argtypes = [I32]
             L.qlora_status_string.restype = ctypes.c_char_p
             L.qlora_version.argtypes = []
@@ -253,6 +259,53 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, Wq: NF4Weight, A: torch.
                                   _ptr(dA), _ptr(dB), gdt, _ptr(workspace), workspace.numel(),
                                   _ptr(d_status), _events(gemm_events), _stream(stream)),
            "qlora_linear_bwd")
+    return dX, dA, dB
+
+
+def qlora_lora_linear_fwd(X: torch.Tensor, W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                          Y: torch.Tensor | None = None, T_save: torch.Tensor | None = None,
+                          workspace: torch.Tensor | None = None, d_status: torch.Tensor | None = None,
+                          gemm_events=None, stream=None) -> torch.Tensor:
+    """qlora_linear_fwd over a dense bf16 weight W [N, K] (plain LoRA)."""
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D bf16 tensor")
+    M, r = X.shape[0], A.shape[0]
+    N, K = W.shape
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(max(qlora_workspace_bytes(M, N, K, r), 16), dtype=torch.uint8, device=X.device)
+    _check(lib().qlora_lora_linear_fwd(_ptr(X), M, _ptr(W), N, K, _ptr(A), _ptr(B), r, float(alpha), _ptr(Y),
+                                       _ptr(T_save), _ptr(workspace), workspace.numel(), _ptr(d_status),
+                                       _events(gemm_events), _stream(stream)), "qlora_lora_linear_fwd")
+    return Y
+
+
+def qlora_lora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, W: torch.Tensor, A: torch.Tensor,
+                          B: torch.Tensor, alpha: float, T_saved: torch.Tensor | None = None,
+                          dX: torch.Tensor | None = None, dA: torch.Tensor | None = None,
+                          dB: torch.Tensor | None = None, grad_dtype=torch.float32, want_dX: bool = True,
+                          workspace: torch.Tensor | None = None, d_status: torch.Tensor | None = None,
+                          gemm_events=None, stream=None):
+    """qlora_linear_bwd over a dense bf16 weight W [N, K] (plain LoRA)."""
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D bf16 tensor")
+    M, r = X.shape[0], A.shape[0]
+    N, K = W.shape
+    dev = X.device
+    if want_dX and dX is None:
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((r, K), dtype=grad_dtype, device=dev)
+    if dB is None:
+        dB = torch.empty((N, r), dtype=grad_dtype, device=dev)
+    gdt = QLORA_F32 if dA.dtype == torch.float32 else QLORA_BF16
+    if workspace is None:
+        workspace = torch.empty(max(qlora_workspace_bytes(M, N, K, r), 16), dtype=torch.uint8, device=dev)
+    _check(lib().qlora_lora_linear_bwd(_ptr(dY), _ptr(X), M, _ptr(W), N, K, _ptr(A), _ptr(B), r, float(alpha),
+                                       _ptr(T_saved), _ptr(dX) if want_dX else None, _ptr(dA), _ptr(dB), gdt,
+                                       _ptr(workspace), workspace.numel(), _ptr(d_status), _events(gemm_events),
+                                       _stream(stream)), "qlora_lora_linear_bwd")
     return dX, dA, dB
 
 

@@ -191,6 +191,35 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M,
                               const qlora_gemm_events* events, void* stream);
 
 /*
+ * The same forward and backward over a dense bf16 weight W [N, K] (plain
+ * LoRA on a 16-bit base), through the same fused GEMM with the weight tile
+ * loaded as is instead of dequantised.  This is the baseline the pages
+ * measure QLoRA against: "QLoRA" (learning-llms page, the fine-print
+ * bullet on wall-clock), "QLoRA" (scalata.ai, "What it costs, and when to
+ * use it": Speed) and katajob.com ("What it costs": step time) all state
+ * that dequantising every layer on every step makes QLoRA steps slower
+ * than plain LoRA on the same model, without a number; timing these two
+ * entries against qlora_linear_fwd / qlora_linear_bwd on the same shapes
+ * gives it.  W is row-major, read only, 16-byte aligned; N % 8 == 0,
+ * K % 64 == 0.  Workspace: qlora_workspace_bytes(M, N, K, r).  Every other
+ * argument, the results' definitions, the error behaviour and the
+ * determinism are those of qlora_linear_fwd / qlora_linear_bwd with W^
+ * replaced by W (every M takes the 2-SM GEMM; T = X A^T is a separate
+ * launch).
+ */
+qlora_status qlora_lora_linear_fwd(const void* X, int64_t M, const void* W, int64_t N,
+                                   int64_t K, const void* A, const void* B, int r,
+                                   float alpha, void* Y, float* T_save, void* workspace,
+                                   size_t ws_bytes, int* d_status,
+                                   const qlora_gemm_events* events, void* stream);
+qlora_status qlora_lora_linear_bwd(const void* dY, const void* X, int64_t M, const void* W,
+                                   int64_t N, int64_t K, const void* A, const void* B, int r,
+                                   float alpha, const float* T_saved, void* dX, void* dA,
+                                   void* dB, qlora_dtype grad_dtype, void* workspace,
+                                   size_t ws_bytes, int* d_status,
+                                   const qlora_gemm_events* events, void* stream);
+
+/*
  * Forward without a caller workspace, for callers that cannot allocate
  * device memory: a plugin host that hands a kernel only its input and
  * output buffers, a process whose device memory is held by another

@@ -137,6 +137,41 @@ def test_linear_bwd_validation():
     assert L.qlora_linear_bwd(*bad) == 1
 
 
+def test_lora_dense_validation():
+    # the dense-bf16 entries apply the NF4 entries' shape rules to (N, K)
+    L = q.lib()
+    M, N, K, r = 16, 256, 512, 8
+    need = q.qlora_workspace_bytes(M, N, K, r)
+    fwd = [FAKE, M, FAKE, N, K, FAKE, FAKE, r, 16.0, FAKE, None, FAKE, need, None, None, None]
+
+    def f(i, v):
+        a = list(fwd); a[i] = v
+        return L.qlora_lora_linear_fwd(*a)
+    assert f(2, None) == 1                  # W
+    assert f(2, FAKE + 8) == 1              # misaligned W
+    assert f(0, None) == 1                  # X
+    assert f(4, 500) == 1                   # K % 64 != 0
+    assert f(3, 252) == 2                   # N % 8 != 0 is not built
+    assert f(1, 0) == 1                     # M
+    assert f(7, 0) == 1 and f(7, 257) == 1  # r
+    assert f(8, float("inf")) == 1          # alpha
+    assert f(12, need - 1) == 6             # workspace too small
+    assert f(11, None) == 6                 # no workspace
+    bwd = [FAKE, FAKE, M, FAKE, N, K, FAKE, FAKE, r, 16.0, None, FAKE, FAKE, FAKE, 0, FAKE, need, None, None,
+           None]
+
+    def b(i, v):
+        a = list(bwd); a[i] = v
+        return L.qlora_lora_linear_bwd(*a)
+    assert b(3, None) == 1                  # W
+    assert b(0, None) == 1                  # dY
+    assert b(12, None) == 1                 # dA
+    assert b(14, 7) == 1                    # grad dtype
+    assert b(5, 96) == 1                    # K % 64 != 0
+    assert b(16, need - 1) == 6
+    assert b(10, FAKE + 4) == 1             # misaligned T_saved
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
