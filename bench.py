@@ -637,6 +637,33 @@ def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_param
                                  "weights": "bf16 copies of the layer's NF4 weights (dequantised)"}
     del Wd
     torch.cuda.empty_cache()
+    # adapter optimiser step (Adam, fp32 master + moments, bf16 copy) over
+    # the adapters of the 32-layer 7B stack: 30 bytes moved per parameter
+    # (read grad, master, m, v; write master, m, v, bf16 copy)
+    wl4 = inputs.STACK7B
+    n_ad = wl4.layers * sum(wl4.r * (N + K) for _, N, K in wl4.shapes)
+    g = torch.Generator(device=dev).manual_seed(4)
+    master = torch.randn(n_ad, generator=g, device=dev) * 0.01
+    mom1 = torch.zeros(n_ad, device=dev)
+    mom2 = torch.zeros(n_ad, device=dev)
+    grad = torch.randn(n_ad, generator=g, device=dev) * 1e-3
+    pbf = torch.empty(n_ad, dtype=torch.bfloat16, device=dev)
+    step_no = [0]
+
+    def adam():
+        step_no[0] += 1
+        q.qlora_adam_step(master, mom1, mom2, grad, step_no[0], 1e-4, weight_decay=0.01, param=pbf,
+                          d_status=layer.status)
+    for _ in range(3):
+        adam()
+    ms = statistics.median(time_events(adam, 10, flush=lambda: l2buf.add_(1)))
+    agbs = 30 * n_ad / (ms * 1e-3) / 1e9
+    out["adam_step"] = {"value": round(agbs, 1), "unit": "GB/s", "params": n_ad, "bytes_per_param": 30,
+                        "us": round(ms * 1e3, 2), "frac_of_hbm": round(agbs / hbm, 4),
+                        "workload": "Adam over the adapters of the 32-layer 7B stack (r = 16)"}
+    assert layer.status.item() == 0, f"device status {layer.status.item()}"
+    del master, mom1, mom2, grad, pbf
+    torch.cuda.empty_cache()
     # decode-shaped forward: 70B MLP weights, M in {1, 4, 16}
     wl = inputs.DECODE
     dec = {}

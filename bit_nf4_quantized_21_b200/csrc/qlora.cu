@@ -25,6 +25,7 @@
 #include "skinny.cuh"
 #include "gemm_nf4_pair.cuh"
 #include "gemv_nf4.cuh"
+#include "adam.cuh"
 
 using namespace qlora;
 
@@ -752,6 +753,44 @@ qlora_status qlora_lora_linear_bwd(const void* dY, const void* X, int64_t M, con
   if (!ensure_smem_attrs()) return QLORA_ERR_CUDA;
   return linear_bwd_core(dY, X, dims_of(M, N, K, r), nullptr, W, A, B, alpha, T_saved, dX, dA, dB, grad_dtype,
                          workspace, d_status, events, static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16, const void* grad,
+                             qlora_dtype grad_dtype, int64_t n, int64_t step, float lr, float beta1, float beta2,
+                             float eps, float weight_decay, float grad_scale, int* d_status, void* stream) {
+  if (n < 0 || step < 1) return QLORA_ERR_INVALID_ARG;
+  if (grad_dtype != QLORA_F32 && grad_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  for (float x : {lr, beta1, beta2, eps, weight_decay, grad_scale})
+    if (!std::isfinite(x)) return QLORA_ERR_INVALID_ARG;
+  if (beta1 < 0.0f || beta1 >= 1.0f || beta2 < 0.0f || beta2 >= 1.0f || eps < 0.0f) return QLORA_ERR_INVALID_ARG;
+  if (n == 0) return QLORA_OK;
+  if (!master || !m || !v || !grad) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(grad)) return QLORA_ERR_INVALID_ARG;
+  if (param_bf16 && !aligned16(param_bf16)) return QLORA_ERR_INVALID_ARG;
+  const double b1t = std::pow(static_cast<double>(beta1), static_cast<double>(step));
+  const double b2t = std::pow(static_cast<double>(beta2), static_cast<double>(step));
+  qlora::AdamArgs a{};
+  a.master = master; a.m = m; a.v = v;
+  a.param = static_cast<__nv_bfloat16*>(param_bf16);
+  a.grad = grad;
+  a.grad_bf16 = grad_dtype == QLORA_BF16 ? 1 : 0;
+  a.n = n;
+  a.grad_scale = grad_scale;
+  a.decay = static_cast<float>(1.0 - static_cast<double>(lr) * static_cast<double>(weight_decay));
+  a.beta1 = beta1;
+  a.one_minus_beta1 = static_cast<float>(1.0 - static_cast<double>(beta1));
+  a.beta2 = beta2;
+  a.one_minus_beta2 = static_cast<float>(1.0 - static_cast<double>(beta2));
+  a.eps = eps;
+  a.step_size = static_cast<float>(static_cast<double>(lr) / (1.0 - b1t));
+  a.rsqrt_bc2 = static_cast<float>(1.0 / std::sqrt(1.0 - b2t));
+  a.status = d_status;
+  const int sms = sm_count();
+  if (sms <= 0) return QLORA_ERR_CUDA;
+  const int64_t want = std::max<int64_t>(1, cdiv(n / 4, qlora::kAdamThreads));
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
+  qlora::k_adam_step<<<grid, qlora::kAdamThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return check_launch();
 }
 
 }  // extern "C"

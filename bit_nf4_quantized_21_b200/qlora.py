@@ -28,6 +28,7 @@ EXPORTED = (
     "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
     "qlora_version", "qlora_linear_fwd_noalloc", "qlora_lora_linear_fwd", "qlora_lora_linear_bwd",
+    "qlora_adam_step",
 )
 
 
@@ -101,6 +102,8 @@ def lib() -> ctypes.CDLL:
             L.qlora_lora_linear_bwd.argtypes = [P, P, I64, P, I64, I64, P, P, I32, F, P, P, P, P, I32, P,
                                                 ctypes.c_size_t, P, P, P]
             L.qlora_lora_linear_bwd.restype = I32
+            L.qlora_adam_step.argtypes = [P, P, P, P, P, I32, I64, I64, F, F, F, F, F, F, P, P]
+            L.qlora_adam_step.restype = I32
             L.qlora_status_string.argtypes = [I32]
             L.qlora_status_string.restype = ctypes.c_char_p
             L.qlora_version.argtypes = []
@@ -307,6 +310,26 @@ def qlora_lora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, W: torch.Tensor, A:
                                        _ptr(workspace), workspace.numel(), _ptr(d_status), _events(gemm_events),
                                        _stream(stream)), "qlora_lora_linear_bwd")
     return dX, dA, dB
+
+
+def qlora_adam_step(master: torch.Tensor, m: torch.Tensor, v: torch.Tensor, grad: torch.Tensor, step: int,
+                    lr: float, betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
+                    param: torch.Tensor | None = None, grad_scale: float = 1.0,
+                    d_status: torch.Tensor | None = None, stream=None) -> None:
+    """One Adam step in place over flat fp32 master/m/v (and an optional bf16
+    copy `param`), with fp32 or bf16 gradients of the same length."""
+    n = master.numel()
+    for t in (m, v, grad) + ((param,) if param is not None else ()):
+        if t.numel() != n:
+            raise ValueError("master, m, v, grad (and param) must have the same number of elements")
+    if master.dtype != torch.float32 or m.dtype != torch.float32 or v.dtype != torch.float32:
+        raise ValueError("master, m and v are fp32")
+    if param is not None and param.dtype != torch.bfloat16:
+        raise ValueError("param is bf16")
+    gdt = QLORA_F32 if grad.dtype == torch.float32 else QLORA_BF16
+    _check(lib().qlora_adam_step(_ptr(master), _ptr(m), _ptr(v), _ptr(param), _ptr(grad), gdt, n, int(step),
+                                 float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay),
+                                 float(grad_scale), _ptr(d_status), _stream(stream)), "qlora_adam_step")
 
 
 def qlora_linear_fwd_noalloc(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor,

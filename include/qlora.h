@@ -220,6 +220,34 @@ qlora_status qlora_lora_linear_bwd(const void* dY, const void* X, int64_t M, con
                                    const qlora_gemm_events* events, void* stream);
 
 /*
+ * One Adam step over a flat array of n adapter parameters ("QLoRA",
+ * infra.bea.ai, "How QLoRA Works", precision table: bf16 adapters and
+ * gradients, Adam state in fp32 at 12 bytes per adapter parameter = an fp32
+ * master copy and the two moments).  The pages print no update rule; this
+ * is Adam as published, with bias correction, and optional decoupled
+ * weight decay (AdamW); per element, fp32, IEEE rounding, in this order:
+ *   g = grad * grad_scale;  theta = master * (1 - lr * weight_decay)
+ *   m = beta1 m + (1 - beta1) g;  v = beta2 v + (1 - beta2) g^2
+ *   master = theta - lr / (1 - beta1^step) * m / (sqrt(v) / sqrt(1 - beta2^step) + eps)
+ *   param_bf16 = bf16_rne(master)            (skipped when NULL)
+ * (the scalar factors are computed on the host in double, then rounded to
+ * fp32).  master, m, v: fp32 [n], updated in place; grad: fp32 or bf16 [n]
+ * (grad_dtype), read only; param_bf16: bf16 [n] or NULL.  Any device
+ * memory the kernel can address works, including managed (pageable)
+ * memory for optimiser state that may be paged out to the host.  All
+ * pointers 16-byte aligned; step >= 1; 0 <= beta1, beta2 < 1; eps >= 0;
+ * finite scalars; n == 0 is a no-op.  A non-finite scaled gradient sets
+ * QLORA_DEV_NONFINITE_BIT in *d_status (if given); results are then
+ * unspecified.  Deterministic.  Use one array layout for all four buffers
+ * (e.g. every projection's A then B, matching its gradient buffer).
+ */
+qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16,
+                             const void* grad, qlora_dtype grad_dtype, int64_t n,
+                             int64_t step, float lr, float beta1, float beta2, float eps,
+                             float weight_decay, float grad_scale, int* d_status,
+                             void* stream);
+
+/*
  * Forward without a caller workspace, for callers that cannot allocate
  * device memory: a plugin host that hands a kernel only its input and
  * output buffers, a process whose device memory is held by another

@@ -23,6 +23,12 @@ only the adapters get gradients; the NF4 base is never updated):
     dB = s dY^T T                    [N, r]
 
 T and G stay unrounded (binary64).  There is no bias: the pages show none.
+
+Adapter optimiser ("QLoRA", infra.bea.ai, "How QLoRA Works", precision
+table: Adam state in fp32, 12 bytes per adapter parameter -- a master copy
+and two moments).  The pages print no update rule; ``adam_step`` is Adam as
+published (Kingma & Ba, moment averages with bias correction) with optional
+decoupled weight decay (Loshchilov & Hutter), in binary64.
 """
 from __future__ import annotations
 
@@ -37,7 +43,7 @@ __all__ = [
     "BLOCK", "GROUP", "load", "build_oracle", "nf4_levels", "f32_to_bf16",
     "bf16_to_f32", "absmax_int_quantize", "nf4_nearest", "nf4_sizes",
     "nf4_quantize", "nf4_dequantize", "linear_fwd", "linear_bwd",
-    "rel_fro", "OracleError",
+    "adam_step", "rel_fro", "OracleError",
 ]
 
 BLOCK = 64
@@ -218,6 +224,22 @@ def linear_bwd(dY, X, W_hat, A, B, alpha: float, r: int, T=None):
     dA = s * (G.T @ X)
     dB = s * (dY.T @ T)
     return {"dX": dX, "dA": dA, "dB": dB, "G": G, "T": T}
+
+
+def adam_step(theta, m, v, g, t: int, lr: float, beta1: float, beta2: float, eps: float,
+              weight_decay: float = 0.0, grad_scale: float = 1.0):
+    """One Adam step at step number t >= 1, in binary64; returns the new
+    (theta, m, v).  Steps in the published order: the decoupled decay of the
+    parameter, the two moment averages, their bias corrections, the update."""
+    theta, m, v = (np.asarray(a, np.float64) for a in (theta, m, v))
+    g = np.asarray(g, np.float64) * float(grad_scale)
+    theta = theta * (1.0 - float(lr) * float(weight_decay))
+    m = float(beta1) * m + (1.0 - float(beta1)) * g
+    v = float(beta2) * v + (1.0 - float(beta2)) * g * g
+    m_hat = m / (1.0 - float(beta1) ** t)
+    v_hat = v / (1.0 - float(beta2) ** t)
+    theta = theta - float(lr) * m_hat / (np.sqrt(v_hat) + float(eps))
+    return theta, m, v
 
 
 def rel_fro(got, ref) -> float:

@@ -361,3 +361,69 @@ def test_linear_backward_is_linear_in_dY():
     g3 = O.linear_bwd(2.0 * dy1 - 0.5 * dy2, X, Wh, A, B, alpha, r)
     for k in ("dX", "dA", "dB"):
         assert np.allclose(g3[k], 2.0 * g1[k] - 0.5 * g2[k], rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- Adam step
+# The pages fix only Adam's precision (fp32 state, 12 bytes per adapter
+# parameter); the update is Adam as published.  Pins: its closed forms and
+# an independent implementation (torch.optim.AdamW in binary64).
+
+def test_adam_first_step_is_signed_step_of_lr():
+    # from zero moments the bias-corrected moments are g and g^2 exactly, so
+    # the first step moves every parameter by lr * g / (|g| + eps)
+    rng = np.random.default_rng(1)
+    theta, g = rng.normal(size=257), rng.normal(size=257) * 1e-3
+    z = np.zeros(257)
+    lr, eps = 1e-3, 1e-8
+    t1, m, v = O.adam_step(theta, z, z, g, 1, lr, 0.9, 0.999, eps)
+    assert np.allclose(t1, theta - lr * g / (np.abs(g) + eps), rtol=0, atol=1e-15)
+    assert np.allclose(m, 0.1 * g, rtol=1e-15) and np.allclose(v, 0.001 * g * g, rtol=1e-12)
+
+
+def test_adam_constant_gradient_moves_linearly():
+    # with a constant gradient the bias corrections undo the averages exactly:
+    # every step is the same lr * g / (|g| + eps)
+    rng = np.random.default_rng(2)
+    theta0, g = rng.normal(size=64), rng.normal(size=64)
+    theta, m, v = theta0, np.zeros(64), np.zeros(64)
+    lr, eps = 2e-3, 1e-6
+    for t in range(1, 11):
+        theta, m, v = O.adam_step(theta, m, v, g, t, lr, 0.8, 0.95, eps)
+    assert np.allclose(theta, theta0 - 10 * lr * g / (np.abs(g) + eps), rtol=0, atol=1e-12)
+
+
+def test_adam_decoupled_decay_alone_is_geometric():
+    theta0 = np.linspace(-2.0, 2.0, 33)
+    theta, m, v = theta0, np.zeros(33), np.zeros(33)
+    lr, wd = 1e-2, 0.1
+    for t in range(1, 6):
+        theta, m, v = O.adam_step(theta, m, v, np.zeros(33), t, lr, 0.9, 0.999, 1e-8, weight_decay=wd)
+    assert np.allclose(theta, theta0 * (1 - lr * wd) ** 5, rtol=1e-14, atol=0)
+
+
+def test_adam_is_gradient_scale_invariant_without_eps():
+    rng = np.random.default_rng(3)
+    theta, g1, g2 = rng.normal(size=50), rng.normal(size=50), rng.normal(size=50)
+    z = np.zeros(50)
+    a = O.adam_step(*O.adam_step(theta, z, z, g1, 1, 1e-3, 0.9, 0.99, 0.0)[:3], g2, 2, 1e-3, 0.9, 0.99, 0.0)
+    b = O.adam_step(*O.adam_step(theta, z, z, g1, 1, 1e-3, 0.9, 0.99, 0.0, grad_scale=64.0)[:3], g2, 2, 1e-3,
+                    0.9, 0.99, 0.0, grad_scale=64.0)
+    assert np.allclose(a[0], b[0], rtol=0, atol=1e-14)
+
+
+def test_adam_matches_torch_adamw_in_binary64():
+    rng = np.random.default_rng(4)
+    n, lr, betas, eps, wd = 300, 3e-3, (0.85, 0.97), 1e-7, 0.05
+    theta0 = rng.normal(size=n)
+    grads = [rng.normal(size=n) for _ in range(6)]
+    p = torch.nn.Parameter(torch.tensor(theta0, dtype=torch.float64))
+    opt = torch.optim.AdamW([p], lr=lr, betas=betas, eps=eps, weight_decay=wd)
+    theta, m, v = theta0, np.zeros(n), np.zeros(n)
+    for t, g in enumerate(grads, start=1):
+        p.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+        theta, m, v = O.adam_step(theta, m, v, g, t, lr, betas[0], betas[1], eps, weight_decay=wd)
+    st = opt.state[p]
+    assert np.allclose(theta, p.detach().numpy(), rtol=0, atol=1e-13)
+    assert np.allclose(m, st["exp_avg"].numpy(), rtol=0, atol=1e-15)
+    assert np.allclose(v, st["exp_avg_sq"].numpy(), rtol=0, atol=1e-15)
