@@ -622,6 +622,21 @@ def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_param
     out["dequantize"] = {"value": round(dgbs, 1), "unit": "GB/s", "shape": [p["N"], p["K"]],
                          "frac_of_hbm": round(dgbs / hbm, 4)}
     del Wout
+    # adapter merge on the gate projection: NF4(W^ + s B A) through an fp32
+    # buffer; bytes moved per weight: NF4 read 0.516 + fp32 write 4 + fp32
+    # read 4 + NF4 write 0.516
+    Wm = torch.empty((p["N"], p["K"]), dtype=torch.float32, device=dev)
+    Wnew = q.empty_nf4(p["N"], p["K"], dev)
+    f = lambda: q.qlora_merge_nf4(p["Wq"], p["A"], p["B"], layer.wl.alpha, out=Wnew, W_merged=Wm,
+                                  d_status=layer.status)
+    for _ in range(3):
+        f()
+    ms = statistics.median(time_events(f, 10, flush=lambda: l2buf.add_(1)))
+    mbytes = 2 * p["Wq"].nbytes() + 8 * p["N"] * p["K"]
+    out["merge"] = {"value": round(mbytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "shape": [p["N"], p["K"]],
+                    "us": round(ms * 1e3, 2), "frac_of_hbm": round(mbytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+    assert layer.status.item() == 0, f"device status {layer.status.item()}"
+    del Wm, Wnew
     # plain LoRA on a bf16 base (the weights' dequantised copies) through the
     # same GEMM, timed with the same harness as the NF4 step beside it: the
     # pages say QLoRA steps are slower than LoRA's without giving a number

@@ -7,7 +7,7 @@ The library is loaded on first use; calls raise if it has not been built.
 """
 from .qlora import (  # noqa: F401
     NF4Weight, QloraError, empty_nf4, lib, qlora_dequantize, qlora_linear_bwd, qlora_linear_fwd,
-    qlora_adam_step, qlora_linear_fwd_noalloc, qlora_lora_linear_bwd, qlora_lora_linear_fwd, qlora_nf4_codebook,
+    qlora_adam_step, qlora_merge_nf4, qlora_linear_fwd_noalloc, qlora_lora_linear_bwd, qlora_lora_linear_fwd, qlora_nf4_codebook,
     qlora_nf4_sizes, qlora_quantize_nf4, qlora_workspace_bytes, status_string,
 )
 

@@ -26,6 +26,7 @@
 #include "gemm_nf4_pair.cuh"
 #include "gemv_nf4.cuh"
 #include "adam.cuh"
+#include "merge.cuh"
 
 using namespace qlora;
 
@@ -791,6 +792,28 @@ qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
   qlora::k_adam_step<<<grid, qlora::kAdamThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return check_launch();
+}
+
+qlora_status qlora_merge_nf4(const qlora_nf4_weight* Wq, const void* A, const void* B, int r, float alpha,
+                             float* W_merged, const qlora_nf4_weight* out, int* d_status, void* stream) {
+  qlora_status st = check_weight(Wq, true);
+  if (st != QLORA_OK) return st;
+  st = check_weight(out, true);
+  if (st != QLORA_OK) return st;
+  if (out->rows != Wq->rows || out->cols != Wq->cols) return QLORA_ERR_INVALID_ARG;
+  if (out->absmax_f32 && !aligned16(out->absmax_f32)) return QLORA_ERR_INVALID_ARG;
+  if (r < 1 || r > 256 || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  if (!A || !B || !W_merged || !aligned16(A) || !aligned16(B) || !aligned16(W_merged)) return QLORA_ERR_INVALID_ARG;
+  const int64_t N = Wq->rows, K = Wq->cols;
+  const float s = alpha / static_cast<float>(r);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int64_t threads = N * (K / 8);
+  qlora::k_merge_nf4<<<static_cast<unsigned>(cdiv(threads, qlora::kMergeThreads)), qlora::kMergeThreads, 0, cs>>>(
+      Wq->codes, Wq->absmax_q8, Wq->group_scale, Wq->absmax_f32, Wq->double_quant, N, K,
+      static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), r, s, W_merged);
+  st = check_launch();
+  if (st != QLORA_OK) return st;
+  return qlora_quantize_nf4(W_merged, QLORA_F32, out, d_status, stream);
 }
 
 }  // extern "C"

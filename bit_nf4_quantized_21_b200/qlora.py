@@ -28,7 +28,7 @@ EXPORTED = (
     "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
     "qlora_version", "qlora_linear_fwd_noalloc", "qlora_lora_linear_fwd", "qlora_lora_linear_bwd",
-    "qlora_adam_step",
+    "qlora_adam_step", "qlora_merge_nf4",
 )
 
 
@@ -104,6 +104,9 @@ def lib() -> ctypes.CDLL:
             L.qlora_lora_linear_bwd.restype = I32
             L.qlora_adam_step.argtypes = [P, P, P, P, P, I32, I64, I64, F, F, F, F, F, F, P, P]
             L.qlora_adam_step.restype = I32
+            L.qlora_merge_nf4.argtypes = [ctypes.POINTER(NF4WeightC), P, P, I32, F, P, ctypes.POINTER(NF4WeightC),
+                                          P, P]
+            L.qlora_merge_nf4.restype = I32
             L.qlora_status_string.argtypes = [I32]
             L.qlora_status_string.restype = ctypes.c_char_p
             L.qlora_version.argtypes = []
@@ -208,6 +211,23 @@ def qlora_quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, double_qua
     _check(lib().qlora_quantize_nf4(_ptr(W), dt, ctypes.byref(cw), _ptr(d_status), _stream(stream)),
            "qlora_quantize_nf4")
     return out
+
+
+def qlora_merge_nf4(Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                    out: NF4Weight | None = None, W_merged: torch.Tensor | None = None,
+                    double_quant: bool = True, d_status: torch.Tensor | None = None, stream=None):
+    """NF4(W^ + (alpha/r) B A) into `out` (new, or Wq itself for in place);
+    returns (out, W_merged) with W_merged the fp32 merged weight."""
+    r = A.shape[0]
+    dev = Wq.codes.device
+    if out is None:
+        out = empty_nf4(Wq.rows, Wq.cols, dev, double_quant)
+    if W_merged is None:
+        W_merged = torch.empty((Wq.rows, Wq.cols), dtype=torch.float32, device=dev)
+    cw, co = Wq.c(), out.c()
+    _check(lib().qlora_merge_nf4(ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha), _ptr(W_merged),
+                                 ctypes.byref(co), _ptr(d_status), _stream(stream)), "qlora_merge_nf4")
+    return out, W_merged
 
 
 def qlora_dequantize(Wq: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

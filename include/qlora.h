@@ -220,6 +220,25 @@ qlora_status qlora_lora_linear_bwd(const void* dY, const void* X, int64_t M, con
                                    const qlora_gemm_events* events, void* stream);
 
 /*
+ * Merge a trained adapter into the frozen base: out = NF4(W^ + s B A),
+ * s = alpha / r ("QLoRA", learning-llms page, the fine-print bullet on
+ * merging: adding the bf16 update into 4-bit weights forces a
+ * re-quantisation; katajob.com, "What it costs": merge friction).  Each
+ * merged weight is formed in fp32, every operation rounded once, in this
+ * order:  acc = 0; for j = 0..r-1: acc = acc + B[n,j] * A[j,k];
+ * W'[n,k] = W^[n,k] + s * acc  (W^ the bf16 dequantised weight), written
+ * to W_merged (fp32 [N, K], caller-provided scratch, left holding W'),
+ * then quantised into `out` exactly as qlora_quantize_nf4 would quantise
+ * W_merged.  A bf16 [r, K], B bf16 [N, r]; 1 <= r <= 256.  `out` has
+ * Wq's rows and cols, its own double_quant setting, and may be Wq itself
+ * (the two launches are ordered on the stream).  Non-finite merged values
+ * set QLORA_DEV_NONFINITE_BIT as in the quantiser.
+ */
+qlora_status qlora_merge_nf4(const qlora_nf4_weight* Wq, const void* A, const void* B, int r,
+                             float alpha, float* W_merged, const qlora_nf4_weight* out,
+                             int* d_status, void* stream);
+
+/*
  * One Adam step over a flat array of n adapter parameters ("QLoRA",
  * infra.bea.ai, "How QLoRA Works", precision table: bf16 adapters and
  * gradients, Adam state in fp32 at 12 bytes per adapter parameter = an fp32

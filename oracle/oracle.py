@@ -43,7 +43,7 @@ __all__ = [
     "BLOCK", "GROUP", "load", "build_oracle", "nf4_levels", "f32_to_bf16",
     "bf16_to_f32", "absmax_int_quantize", "nf4_nearest", "nf4_sizes",
     "nf4_quantize", "nf4_dequantize", "linear_fwd", "linear_bwd",
-    "adam_step", "rel_fro", "OracleError",
+    "adam_step", "merge_nf4", "rel_fro", "OracleError",
 ]
 
 BLOCK = 64
@@ -224,6 +224,25 @@ def linear_bwd(dY, X, W_hat, A, B, alpha: float, r: int, T=None):
     dA = s * (G.T @ X)
     dB = s * (dY.T @ T)
     return {"dX": dX, "dA": dA, "dB": dB, "G": G, "T": T}
+
+
+def merge_nf4(q: dict, A, B, alpha: float, r: int) -> np.ndarray:
+    """The merged weight W^ + s B A as fp32 [N, K], before re-quantisation
+    ("QLoRA", learning-llms page, the fine-print bullet on merging: adding
+    the bf16 update into 4-bit weights forces a re-quantisation).  The pages
+    fix no precision for it; the merged values decide integer codes, so this
+    takes the library's precision and order: fp32, every operation rounded
+    once, acc = sum over j of B[:, j] * A[j, :] in j order, then W^ + s acc
+    with s = fp32(alpha) / fp32(r).  numpy float32 arithmetic rounds each
+    operation (no fused multiply-add)."""
+    W = bf16_to_f32(nf4_dequantize(q)).astype(np.float32)
+    a = bf16_to_f32(np.asarray(A, np.uint16)).astype(np.float32)
+    b = bf16_to_f32(np.asarray(B, np.uint16)).astype(np.float32)
+    s = np.float32(alpha) / np.float32(r)
+    acc = np.zeros(W.shape, np.float32)
+    for j in range(r):
+        acc = acc + b[:, j:j + 1] * a[j:j + 1, :]
+    return W + s * acc
 
 
 def adam_step(theta, m, v, g, t: int, lr: float, beta1: float, beta2: float, eps: float,

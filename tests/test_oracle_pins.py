@@ -427,3 +427,37 @@ def test_adam_matches_torch_adamw_in_binary64():
     assert np.allclose(theta, p.detach().numpy(), rtol=0, atol=1e-13)
     assert np.allclose(m, st["exp_avg"].numpy(), rtol=0, atol=1e-15)
     assert np.allclose(v, st["exp_avg_sq"].numpy(), rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------- adapter merge
+
+def _int_adapters(N, K, r, seed):
+    """Small-integer adapters: every product and partial sum is exact in fp32."""
+    rng = np.random.default_rng(seed)
+    A = rng.integers(-4, 5, size=(r, K)).astype(np.float32)
+    B = rng.integers(-4, 5, size=(N, r)).astype(np.float32)
+    return O.f32_to_bf16(A), O.f32_to_bf16(B), A.astype(np.float64), B.astype(np.float64)
+
+
+def test_merge_with_zero_adapter_is_the_dequantised_weight():
+    rng = np.random.default_rng(21)
+    W = (rng.normal(size=(16, 256)) * 0.02).astype(np.float32)
+    q = O.nf4_quantize(W)
+    r = 8
+    A = O.f32_to_bf16(rng.normal(size=(r, 256)).astype(np.float32))
+    Bz = np.zeros((16, r), np.uint16)
+    merged = O.merge_nf4(q, A, Bz, 16.0, r)
+    assert np.array_equal(merged, O.bf16_to_f32(O.nf4_dequantize(q)))
+
+
+def test_merge_of_a_zero_weight_is_the_exact_adapter_product():
+    # a zero weight dequantises to exact zeros (all codes 7), so with integer
+    # adapters the merged weight is s (B A) exactly; B A is not symmetric, so
+    # a transposed operand or a wrong index fails
+    N, K, r = 24, 192, 8
+    q = O.nf4_quantize(np.zeros((N, K), np.float32))
+    A, B, a, b = _int_adapters(N, K, r, seed=22)
+    merged = O.merge_nf4(q, A, B, 2.0 * r, r)
+    assert np.array_equal(merged.astype(np.float64), 2.0 * (b @ a))
+    merged = O.merge_nf4(q, A, B, 0.5 * r, r)       # s = 0.5
+    assert np.array_equal(merged.astype(np.float64), 0.5 * (b @ a))
