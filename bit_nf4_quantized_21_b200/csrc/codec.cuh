@@ -12,79 +12,86 @@ namespace qlora {
 
 constexpr int kQuantThreads = 256;  // one CTA per 256-block group
 
-template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
-
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+// The 8 weights a thread holds per block, kept as loaded (a bf16 uint4
+// is 4 registers instead of 8 floats) and widened only when encoded.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> { uint4 u; };
+template <> struct Raw8<float> { float4 a, b; };
+__device__ __forceinline__ Raw8<__nv_bfloat16> load_raw8(const __nv_bfloat16* p) {
+  return {__ldg(reinterpret_cast<const uint4*>(p))};
+}
+__device__ __forceinline__ Raw8<float> load_raw8(const float* p) {
+  return {__ldg(reinterpret_cast<const float4*>(p)), __ldg(reinterpret_cast<const float4*>(p) + 1)};
+}
+__device__ __forceinline__ void widen8(const Raw8<__nv_bfloat16>& r, float (&v)[8]) {
+  const uint32_t w[4] = {r.u.x, r.u.y, r.u.z, r.u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     v[2 * i] = __uint_as_float(w[i] << 16);
     v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
 }
-
-template <>
-__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+__device__ __forceinline__ void widen8(const Raw8<float>& r, float (&v)[8]) {
+  v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
+  v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
 }
 
-// Nearest NF4 level of a normalised weight: code = #{i : x > t_i}, found by a
-// 4-step binary search over the 15 sorted thresholds; the first step's
-// threshold (t_7) comes from a register, the other three from shared memory.
-__device__ __forceinline__ uint32_t nf4_encode(float x, const float* s_thr, float t7) {
-  uint32_t c = (x > t7) ? 8u : 0u;
-  c += (x > s_thr[c + 3]) ? 4u : 0u;
-  c += (x > s_thr[c + 1]) ? 2u : 0u;
-  c += (x > s_thr[c]) ? 1u : 0u;
-  return c;
+// Nearest NF4 level of a normalised weight: code = #{i : x > t_i}, from the
+// cell table (nf4_constants.cuh): cell = rint(32 x + 32.5), found with one
+// fused multiply-add and the 1.5 * 2^23 rounding trick (the sum's low
+// mantissa bits are the integer), then one compare against the cell's
+// threshold.  The index is clamped to the table (a NaN x, from a block with
+// an infinite absmax, reads the last cell; such blocks are flagged).
+__device__ __forceinline__ uint32_t nf4_encode(float x, const uint2* s_cell) {
+  const float y = __fadd_rn(__fmaf_rn(x, 32.0f, 32.5f), 12582912.0f);
+  const uint32_t idx = min(static_cast<uint32_t>(__float_as_int(y)) - 0x4B400000u, 65u);
+  const uint2 e = s_cell[idx];
+  return e.y + ((x > __uint_as_float(e.x)) ? 1u : 0u);
 }
 
 // K1.  Grid: one CTA per group of 256 blocks (16384 weights).  Eight threads
 // share a 64-weight block (8 weights each, one 16-byte load of bf16), so a
 // warp reads 4 whole blocks = 512 contiguous bytes and writes 128 contiguous
 // bytes of codes.  The block absmax is a warp-shuffle max over the 8 lanes.
-// All 8 of a thread's loads are issued before any is used, so every thread
-// keeps 8 x 16 B in flight (HBM needs tens of KB per SM in flight).
+// All 8 of a thread's loads are issued before any is used and are kept as
+// loaded (32 registers for bf16), which leaves room for 5 CTAs per SM: with
+// 8 x 16 B in flight per thread that is 160 KB per SM (HBM needs tens of KB
+// per SM in flight).  The encoding is ~11 instructions per weight.
 template <typename T>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, sizeof(T) == 2 ? 5 : 3)
     k_quantize_nf4(const T* __restrict__ w, int64_t nblocks, int dq, uint8_t* __restrict__ codes,
                    uint8_t* __restrict__ q8, float* __restrict__ s2,
                    float* __restrict__ absmax_out, int* status) {
-  __shared__ float s_thr[16];
+  __shared__ uint2 s_cell[66];
   __shared__ float s_absmax[256];
   __shared__ float s_wmax[kQuantThreads / 32];
   const int tid = threadIdx.x;
-  if (tid < 15) s_thr[tid] = c_nf4_threshold[tid];
-  __syncthreads();
+  if (tid < 66) s_cell[tid] = make_uint2(__float_as_uint(c_nf4_cells.c[tid].thr), c_nf4_cells.c[tid].base);
 
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * 256;
   const int nb = static_cast<int>((nblocks - b0) < 256 ? (nblocks - b0) : 256);
   const int sub = tid & 7;
-  const float t7 = c_nf4_threshold[7];
   bool nonfinite = false;
 
-  float v[8][8];
+  Raw8<T> raw[8];
 #pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int lb = it * 32 + (tid >> 3);
-    if (lb < nb) load8<T>(w + (b0 + lb) * 64 + sub * 8, v[it]);
+    if (lb < nb) raw[it] = load_raw8(w + (b0 + lb) * 64 + sub * 8);
   }
+  __syncthreads();   // the cell table is in shared memory
 #pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int lb = it * 32 + (tid >> 3);
     const bool valid = lb < nb;
     const int64_t b = b0 + lb;
+    float v[8];
+    widen8(raw[it], v);
     uint32_t mbits = 0;
     if (valid) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mbits = max(mbits, __float_as_uint(v[it][i]) & 0x7FFFFFFFu);
+      for (int i = 0; i < 8; ++i) mbits = max(mbits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
     }
     // max over the 8 lanes of the block (integer order = magnitude order,
     // with inf/NaN patterns above every finite value)
@@ -101,7 +108,7 @@ __global__ void __launch_bounds__(kQuantThreads)
       const float inv = __frcp_rn(absmax);
       word = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) word |= nf4_encode(__fmul_rn(v[it][i], inv), s_thr, t7) << (4 * i);
+      for (int i = 0; i < 8; ++i) word |= nf4_encode(__fmul_rn(v[i], inv), s_cell) << (4 * i);
     }
     reinterpret_cast<uint32_t*>(codes)[b * 8 + sub] = word;
     if (sub == 0) s_absmax[lb] = absmax;
