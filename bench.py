@@ -823,10 +823,36 @@ def run_only(args):
     """One projection's forward or backward call, repeated: the small case
     for kernel profiles (ncu) of the fused GEMM; with --only decode, the
     decode-shaped forward of one 70B MLP matrix (--proj 0: 28672 x 8192,
-    1: 8192 x 28672) at --tokens <= 16."""
+    1: 8192 x 28672) at --tokens <= 16; with --only quantize, the quantiser
+    over the seven LLaMA-7B projections (bf16), --steps repetitions."""
     import bit_nf4_quantized_21_b200 as q
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    if args.only == "quantize":
+        Ws, outs = [], []
+        for i, (name, N, K) in enumerate(WL.shapes):
+            Ws.append(inputs.weight((N, K), WL.w_std, inputs.matrix_seed(WL.base_seed, 0, i), device=dev))
+            outs.append(q.empty_nf4(N, K, dev))
+        l2 = torch.empty(L2_BYTES // 2, dtype=torch.float32, device=dev)
+        params = sum(w.numel() for w in Ws)
+        res = []
+        for rep in range(args.steps):
+            l2.add_(1)
+            torch.cuda._sleep(2_000_000)
+            evs = []
+            for W, o in zip(Ws, outs):
+                e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                e[0].record()
+                q.qlora_quantize_nf4(W, out=o)
+                e[1].record()
+                evs.append(e)
+            torch.cuda.synchronize()
+            if rep >= 1:
+                res.append(sum(a.elapsed_time(b) for a, b in evs))
+        ms = statistics.median(res)
+        print(json.dumps({"only": "quantize", "params": params, "ms": round(ms, 4),
+                          "GBps": round(params * 2.516 / (ms * 1e-3) / 1e9, 1)}), flush=True)
+        return
     if args.only == "decode":
         wl = inputs.DECODE
         name, N, K = wl.shapes[args.proj]
@@ -892,7 +918,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--only", choices=("gemm-fwd", "gemm-dx", "decode"), default=None,
+    ap.add_argument("--only", choices=("gemm-fwd", "gemm-dx", "decode", "quantize"), default=None,
                     help="profile mode: repeat one projection's call (see --proj, --tokens)")
     ap.add_argument("--proj", type=int, default=4)
     ap.add_argument("--tokens", type=int, default=2048)
