@@ -26,11 +26,15 @@
  *     asynchronously on `stream`.  No call allocates memory, synchronises, or
  *     keeps state between calls.
  *   - `d_status` (nullable) is a device int the kernels OR error bits into:
- *     QLORA_DEV_NONFINITE_BIT (non-finite weight seen by the quantiser) and
+ *     QLORA_DEV_NONFINITE_BIT (a non-finite weight seen by the quantiser or
+ *     the merge, or a non-finite gradient seen by the Adam step) and
  *     QLORA_DEV_TIMEOUT_BIT (a pipeline wait gave up after ~2 s; the kernel
  *     then returns early and its outputs are unspecified).  The caller zeroes
  *     it and reads it after synchronising.
- *   - Errors: a call that returns anything but QLORA_OK has enqueued nothing.
+ *   - Errors: a call that returns a validation error (anything but QLORA_OK
+ *     and QLORA_ERR_CUDA) has enqueued nothing.  QLORA_ERR_CUDA means a
+ *     launch or tensor-map call failed; launches the same call had already
+ *     enqueued may still run, and its outputs are unspecified.
  */
 #ifndef QLORA_H
 #define QLORA_H
