@@ -73,10 +73,13 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, log_dir: str | None = None):
+        """Samples go to <log_dir>/clocks_rank<index>.csv (the system's
+        temporary directory when no log_dir is given)."""
+        import tempfile
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = os.path.join(log_dir or tempfile.gettempdir(), f"clocks_rank{index}.csv")
 
     def start(self):
         try:
@@ -366,7 +369,7 @@ def run_ours(args):
                 for _ in range(2 * nproj)] for _ in range(args.steps)]
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, args.clock_log)
     clocks.start()
     time.sleep(0.3)
     barrier()
@@ -918,6 +921,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--clock-log", default=None,
+                    help="directory for the raw nvidia-smi clock samples (default: the temporary directory)")
     ap.add_argument("--only", choices=("gemm-fwd", "gemm-dx", "decode", "quantize"), default=None,
                     help="profile mode: repeat one projection's call (see --proj, --tokens)")
     ap.add_argument("--proj", type=int, default=4)
