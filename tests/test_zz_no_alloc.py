@@ -37,7 +37,10 @@ def _call_noalloc(X, Wq, A, B, alpha, Y, T):
     return rc
 
 
-@pytest.mark.parametrize("M,N,K,r", [(200, 264, 576, 8), (2048, 4096, 4096, 16), (96, 136, 448, 5)])
+@pytest.mark.parametrize("M,N,K,r", [
+    (200, 264, 576, 8), (2048, 4096, 4096, 16), (96, 136, 448, 5),
+    (16, 512, 1024, 16), (1, 256, 512, 8),      # decode shapes: the weight-streaming kernel on the fixed scratch
+])
 def test_noalloc_forward_matches_workspace_forward_twice(M, N, K, r):
     alpha = 2.0 * r
     for call, seed in enumerate((101, 202)):          # two calls in a row, different inputs
