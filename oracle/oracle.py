@@ -33,6 +33,7 @@ decoupled weight decay (Loshchilov & Hutter), in binary64.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 import threading
@@ -43,7 +44,8 @@ __all__ = [
     "BLOCK", "GROUP", "load", "build_oracle", "nf4_levels", "f32_to_bf16",
     "bf16_to_f32", "absmax_int_quantize", "nf4_nearest", "nf4_sizes",
     "nf4_quantize", "nf4_dequantize", "linear_fwd", "linear_bwd",
-    "adam_step", "merge_nf4", "rel_fro", "OracleError",
+    "adam_step", "merge_nf4", "philox4x64_10", "philox4x64_10_blocks", "dropout_threshold",
+    "lora_dropout_keep", "linear_fwd_dropout", "linear_bwd_dropout", "rel_fro", "OracleError",
 ]
 
 BLOCK = 64
@@ -243,6 +245,107 @@ def merge_nf4(q: dict, A, B, alpha: float, r: int) -> np.ndarray:
     for j in range(r):
         acc = acc + b[:, j:j + 1] * a[j:j + 1, :]
     return W + s * acc
+
+
+# ---------------------------------------------------------------- LoRA dropout
+# The infra.bea.ai "QLoRA" page, §3 "Implementation", configures the
+# adapters with lora_dropout = 0.05 (a PEFT LoraConfig) without defining it.
+# Reading: inverted dropout on the adapter's input X -- each element kept
+# with probability 1 - p, kept elements scaled by 1/(1 - p) -- with one mask
+# per call drawn from a counter-based generator, so that a kernel can
+# regenerate it anywhere.  Because X * keep is still exactly bf16, the
+# 1/(1 - p) is applied to the fp32 products (T, dA, and dX's adapter term).
+#
+# Generator: Philox-4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random
+# numbers: as easy as 1, 2, 3", SC 2011): 10 rounds of two 64x64 -> 128-bit
+# products on a 4-word counter with a 2-word key bumped by two Weyl
+# constants after every round.
+
+_PHILOX_M = (0xD2E7470EE14C6C93, 0xCA5A826395121157)   # round multipliers
+_PHILOX_W = (0x9E3779B97F4A7C15, 0xBB67AE8584CAA73B)   # key increments (Weyl)
+_U64 = (1 << 64) - 1
+
+
+def philox4x64_10(counter, key):
+    """One Philox-4x64-10 block: 4 words out of a 4-word counter and a 2-word
+    key (Python integers, the definition written out)."""
+    c0, c1, c2, c3 = (int(x) & _U64 for x in counter)
+    k0, k1 = (int(x) & _U64 for x in key)
+    for _ in range(10):
+        p0, p1 = _PHILOX_M[0] * c0, _PHILOX_M[1] * c2
+        c0, c1, c2, c3 = ((p1 >> 64) ^ c1 ^ k0) & _U64, p1 & _U64, ((p0 >> 64) ^ c3 ^ k1) & _U64, p0 & _U64
+        k0, k1 = (k0 + _PHILOX_W[0]) & _U64, (k1 + _PHILOX_W[1]) & _U64
+    return c0, c1, c2, c3
+
+
+def _mulhilo64(a: np.ndarray, b: int):
+    """(high, low) 64-bit halves of a * b for uint64 arrays a, from 32-bit parts."""
+    m32 = np.uint64(0xFFFFFFFF)
+    a = a.astype(np.uint64)
+    al, ah = a & m32, a >> np.uint64(32)
+    bl, bh = np.uint64(b & 0xFFFFFFFF), np.uint64(b >> 32)
+    p0, p1, p2, p3 = al * bl, al * bh, ah * bl, ah * bh
+    mid = (p0 >> np.uint64(32)) + (p1 & m32) + (p2 & m32)
+    hi = p3 + (p1 >> np.uint64(32)) + (p2 >> np.uint64(32)) + (mid >> np.uint64(32))
+    lo = (mid << np.uint64(32)) | (p0 & m32)
+    return hi, lo
+
+
+def philox4x64_10_blocks(c0: np.ndarray, key):
+    """Philox-4x64-10 of counters (c0[i], 0, 0, 0) under one key, vectorised
+    over i; returns a [len(c0), 4] uint64 array.  Same rounds as the scalar
+    definition above."""
+    with np.errstate(over="ignore"):
+        x0 = np.asarray(c0, np.uint64)
+        x1 = np.zeros_like(x0); x2 = np.zeros_like(x0); x3 = np.zeros_like(x0)
+        k0, k1 = int(key[0]) & _U64, int(key[1]) & _U64
+        for _ in range(10):
+            h0, l0 = _mulhilo64(x0, _PHILOX_M[0])
+            h1, l1 = _mulhilo64(x2, _PHILOX_M[1])
+            x0, x1, x2, x3 = h1 ^ x1 ^ np.uint64(k0), l1, h0 ^ x3 ^ np.uint64(k1), l0
+            k0, k1 = (k0 + _PHILOX_W[0]) & _U64, (k1 + _PHILOX_W[1]) & _U64
+    return np.stack([x0, x1, x2, x3], axis=1)
+
+
+def dropout_threshold(p: float) -> int:
+    """Integer cut: an element is dropped when the top 32 bits of its word are
+    below ceil(p * 2^32) (exact: scaling by 2^32 is exact in binary64)."""
+    if not 0.0 <= p < 1.0:
+        raise ValueError("dropout p must be in [0, 1)")
+    return int(math.ceil(float(p) * 4294967296.0))
+
+
+def lora_dropout_keep(seed: int, M: int, K: int, p: float) -> np.ndarray:
+    """Keep mask [M, K] of one call: element e = m K + k takes word e % 4 of
+    Philox-4x64-10 at counter (e // 4, 0, 0, 0), key (seed, 0), and is kept
+    when that word's top 32 bits are >= dropout_threshold(p)."""
+    n = M * K
+    words = philox4x64_10_blocks(np.arange((n + 3) // 4, dtype=np.uint64), (seed, 0)).reshape(-1)[:n]
+    return ((words >> np.uint64(32)) >= np.uint64(dropout_threshold(p))).reshape(M, K)
+
+
+def linear_fwd_dropout(X, W_hat, A, B, alpha: float, r: int, keep: np.ndarray, p: float):
+    """Forward with dropout on the adapter input, binary64: T = (X * keep) A^T
+    / (1 - p); Y = X W^T + s T B^T (the frozen path sees X undropped)."""
+    X, W, A, B = _f64(X), _f64(W_hat), _f64(A), _f64(B)
+    s = float(alpha) / float(r)
+    T = ((X * keep) @ A.T) / (1.0 - float(p))
+    Y = X @ W.T + s * (T @ B.T)
+    return Y, T
+
+
+def linear_bwd_dropout(dY, X, W_hat, A, B, alpha: float, r: int, keep: np.ndarray, p: float, T=None):
+    """Backward of linear_fwd_dropout for the same mask, binary64: G = dY B;
+    dX = dY W^ + s (G A) * keep / (1 - p); dA = s G^T (X * keep) / (1 - p);
+    dB = s dY^T T."""
+    dY, X, A, B = _f64(dY), _f64(X), _f64(A), _f64(B)
+    s = float(alpha) / float(r)
+    q = 1.0 - float(p)
+    Xk = X * keep
+    T = (Xk @ A.T) / q if T is None else np.asarray(T, np.float64)
+    G = dY @ B
+    dX = None if W_hat is None else dY @ _f64(W_hat) + s * ((G @ A) * keep) / q
+    return {"dX": dX, "dA": s * (G.T @ Xk) / q, "dB": s * (dY.T @ T), "G": G}
 
 
 def adam_step(theta, m, v, g, t: int, lr: float, beta1: float, beta2: float, eps: float,

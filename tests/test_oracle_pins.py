@@ -461,3 +461,81 @@ def test_merge_of_a_zero_weight_is_the_exact_adapter_product():
     assert np.array_equal(merged.astype(np.float64), 2.0 * (b @ a))
     merged = O.merge_nf4(q, A, B, 0.5 * r, r)       # s = 0.5
     assert np.array_equal(merged.astype(np.float64), 0.5 * (b @ a))
+
+
+# --------------------------------------------------------------- LoRA dropout
+
+def test_philox_matches_numpy_philox():
+    # numpy's Philox (an independent implementation of Philox-4x64-10)
+    # increments its 256-bit counter before each block, so its counter
+    # c - 1 produces our block at counter c
+    rng = np.random.default_rng(31)
+    for _ in range(20):
+        c = [int(rng.integers(1, 1 << 62)), int(rng.integers(0, 1 << 62)), int(rng.integers(0, 1 << 62)),
+             int(rng.integers(0, 1 << 62))]
+        k = [int(rng.integers(0, 1 << 62)), int(rng.integers(0, 1 << 62))]
+        bg = np.random.Philox(key=np.array(k, dtype=np.uint64),
+                              counter=np.array([c[0] - 1, c[1], c[2], c[3]], dtype=np.uint64))
+        assert tuple(int(x) for x in bg.random_raw(4)) == O.philox4x64_10(c, k)
+
+
+def test_philox_blocks_match_scalar_definition():
+    rng = np.random.default_rng(32)
+    c0 = rng.integers(0, 1 << 63, size=64, dtype=np.uint64)
+    key = (int(rng.integers(0, 1 << 63)), int(rng.integers(0, 1 << 63)))
+    got = O.philox4x64_10_blocks(c0, key)
+    for i in range(64):
+        assert tuple(int(x) for x in got[i]) == O.philox4x64_10((int(c0[i]), 0, 0, 0), key)
+
+
+def test_dropout_cut_and_keep_rate():
+    assert O.dropout_threshold(0.0) == 0
+    assert O.dropout_threshold(0.5) == 1 << 31
+    assert O.dropout_threshold(0.05) == 214748365          # ceil(0.05 * 2^32) = ceil(214748364.8)
+    for p in (0.05, 0.5):
+        keep = O.lora_dropout_keep(11, 512, 2048, p)
+        n = keep.size
+        sigma = math.sqrt(n * p * (1 - p))
+        assert abs(keep.sum() - n * (1 - p)) <= 5 * sigma
+    assert O.lora_dropout_keep(11, 64, 128, 0.0).all()
+
+
+def test_dropout_mask_is_per_element_and_seeded():
+    a = O.lora_dropout_keep(5, 40, 192, 0.3)
+    b = O.lora_dropout_keep(5, 45, 192, 0.3)               # a taller matrix: same first rows
+    assert np.array_equal(a, b[:40])
+    flat = O.lora_dropout_keep(5, 1, 40 * 192, 0.3)        # element e = m K + k, whatever the shape
+    assert np.array_equal(a.reshape(-1), flat.reshape(-1))
+    assert not np.array_equal(a, O.lora_dropout_keep(6, 40, 192, 0.3))
+
+
+def test_dropout_layer_without_dropout_is_the_plain_layer():
+    X, Wh, A, B, dY, alpha, r = _small_problem(seed=41)
+    keep = np.ones((X.shape[0], X.shape[1]), bool)
+    Y0, T0 = O.linear_fwd(X, Wh, A, B, alpha, r)
+    Y1, T1 = O.linear_fwd_dropout(X, Wh, A, B, alpha, r, keep, 0.0)
+    assert np.allclose(Y1, Y0, rtol=1e-14, atol=1e-14) and np.allclose(T1, T0, rtol=1e-14, atol=1e-14)
+    g0 = O.linear_bwd(dY, X, Wh, A, B, alpha, r)
+    g1 = O.linear_bwd_dropout(dY, X, Wh, A, B, alpha, r, keep, 0.0)
+    for k in ("dX", "dA", "dB"):
+        assert np.allclose(g1[k], g0[k], rtol=1e-13, atol=1e-13)
+
+
+def test_dropout_layer_gradients_by_central_differences():
+    # with the mask fixed the layer is linear in X, A and B, so for the loss
+    # L = <dY, Y> a central difference along any direction is exact up to
+    # rounding; it checks every term of dX, dA, dB (mask, 1/(1-p), s)
+    X, Wh, A, B, dY, alpha, r = _small_problem(seed=42)
+    x, a, b, dy = (O.bf16_to_f32(t).astype(np.float64) for t in (X, A, B, dY))
+    p = 0.3
+    keep = O.lora_dropout_keep(9, x.shape[0], x.shape[1], p)
+    g = O.linear_bwd_dropout(dy, x, Wh, a, b, alpha, r, keep, p)
+    loss = lambda xx, aa, bb: float(np.sum(dy * O.linear_fwd_dropout(xx, Wh, aa, bb, alpha, r, keep, p)[0]))
+    rng = np.random.default_rng(43)
+    h = 1e-3
+    for name, base, grad in (("dX", x, g["dX"]), ("dA", a, g["dA"]), ("dB", b, g["dB"])):
+        D = rng.normal(size=base.shape)
+        args = {"dX": lambda e: (x + e * D, a, b), "dA": lambda e: (x, a + e * D, b),
+                "dB": lambda e: (x, a, b + e * D)}[name]
+        fd = (loss(*args(h)) - loss(*args(-h))) / (2 * h)
+        assert abs(fd - float(np.sum(grad * D))) <= 1e-8 * max(1.0, abs(fd)), name
