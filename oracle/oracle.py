@@ -44,7 +44,8 @@ __all__ = [
     "BLOCK", "GROUP", "load", "build_oracle", "nf4_levels", "f32_to_bf16",
     "bf16_to_f32", "absmax_int_quantize", "nf4_nearest", "nf4_sizes",
     "nf4_quantize", "nf4_dequantize", "linear_fwd", "linear_bwd",
-    "adam_step", "merge_nf4", "philox4x64_10", "philox4x64_10_blocks", "dropout_threshold",
+    "adam_step", "merge_nf4", "e4m3_values", "e4m3_encode", "nf4_quantize_fp8", "nf4_dequantize_fp8",
+    "philox4x64_10", "philox4x64_10_blocks", "dropout_threshold",
     "lora_dropout_keep", "linear_fwd_dropout", "linear_bwd_dropout", "rel_fro", "OracleError",
 ]
 
@@ -245,6 +246,75 @@ def merge_nf4(q: dict, A, B, alpha: float, r: int) -> np.ndarray:
     for j in range(r):
         acc = acc + b[:, j:j + 1] * a[j:j + 1, :]
     return W + s * acc
+
+
+# ------------------------------------------------ FP8 second-level scales
+# "QLoRA" (infra.bea.ai), §1 "Double Quantization": the fp32 block scales are
+# themselves quantised "to FP8" (0.125 bits per weight).  Reading: FP8 E4M3
+# (bias 7, 3 mantissa bits, largest finite 448, code 0x7F is NaN), one fp32
+# scale per group of 256 blocks s2 = fp32(m / 448) with m the group's
+# largest absmax, q = E4M3 round-to-nearest-even, saturating at 448, of
+# fp32(absmax / s2); m < FLT_MIN gives s2 = 0 and q = 0.  The NF4 codes come
+# from the fp32 absmax as in the 8-bit format; dequantisation uses
+# absmax' = fp32(E4M3(q) * s2).  (The QLoRA paper also subtracts the group
+# mean first; the pages do not, so neither does this reading.)
+
+def e4m3_values() -> np.ndarray:
+    """The 127 non-negative finite E4M3 values, by code 0..126."""
+    v = []
+    for code in range(127):
+        e, m = code >> 3, code & 7
+        v.append((m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.array(v, np.float64)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 codes of non-negative values: nearest value, ties to the even
+    code, values above 448 saturate to 448 (code 126).  Brute force over the
+    codebook (the codes are sorted by value)."""
+    vals = e4m3_values()
+    x = np.asarray(x, np.float64).reshape(-1)
+    if np.any(~np.isfinite(x)) or np.any(x < 0):
+        raise ValueError("e4m3_encode takes finite non-negative values")
+    d = np.abs(x[:, None] - vals[None, :])
+    best = d.min(axis=1, keepdims=True)
+    ties = d == best
+    codes = np.arange(127)
+    # among the nearest, the even code (two values can tie; their codes are adjacent)
+    pick = np.where(ties & (codes[None, :] % 2 == 0), codes[None, :], 1000).min(axis=1)
+    pick = np.where(pick == 1000, np.argmax(ties, axis=1), pick)
+    return np.minimum(pick, 126).astype(np.uint8)
+
+
+def nf4_quantize_fp8(w: np.ndarray) -> dict:
+    """NF4 codes with FP8 (E4M3) second-level scales: codes and fp32 absmax
+    from the C quantiser, then the group scales and E4M3 codes as above."""
+    base = nf4_quantize(w, double_quant=False)
+    a = base["absmax"].astype(np.float32)
+    n = a.size
+    groups = (n + GROUP - 1) // GROUP
+    s2 = np.zeros(groups, np.float32)
+    q = np.zeros(n, np.uint8)
+    for g in range(groups):
+        blk = a[g * GROUP:(g + 1) * GROUP]
+        m = np.float32(blk.max())
+        if not m >= np.float32(np.finfo(np.float32).tiny):
+            continue
+        s2[g] = np.float32(m) / np.float32(448.0)
+        q[g * GROUP:(g + 1) * GROUP] = e4m3_encode(blk / s2[g])
+    return {"codes": base["codes"], "absmax": base["absmax"], "q8": q, "s2": s2,
+            "rows": base["rows"], "cols": base["cols"], "fp8": True}
+
+
+def nf4_dequantize_fp8(q: dict) -> np.ndarray:
+    """bf16 bits of the dequantised weight under FP8 scales: absmax' =
+    fp32(E4M3(q) * s2) per block, then bf16(level * absmax') as for the
+    fp32-absmax format."""
+    vals = e4m3_values().astype(np.float32)
+    s2 = np.repeat(q["s2"], GROUP)[:q["q8"].size]
+    absmax = (vals[q["q8"]] * s2).astype(np.float32)
+    return nf4_dequantize({"codes": q["codes"], "absmax": absmax, "rows": q["rows"], "cols": q["cols"],
+                           "double_quant": False})
 
 
 # ---------------------------------------------------------------- LoRA dropout

@@ -539,3 +539,57 @@ def test_dropout_layer_gradients_by_central_differences():
                 "dB": lambda e: (x, a, b + e * D)}[name]
         fd = (loss(*args(h)) - loss(*args(-h))) / (2 * h)
         assert abs(fd - float(np.sum(grad * D))) <= 1e-8 * max(1.0, abs(fd)), name
+
+
+# ------------------------------------------------ FP8 second-level scales
+
+def test_e4m3_encoder_matches_torch_float8():
+    # torch's float8_e4m3fn conversion (independent) rounds to nearest even;
+    # it agrees with the saturating encoder everywhere up to 464
+    vals = O.e4m3_values()
+    mids = (vals[1:] + vals[:-1]) / 2
+    rng = np.random.default_rng(51)
+    x = np.concatenate([vals, mids, np.nextafter(mids, 0), np.nextafter(mids, 1e9),
+                        rng.uniform(0, 460, 2000), rng.uniform(0, 1e-2, 500)]).astype(np.float32)
+    x = x[x <= 460]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(x), ref)
+
+
+def test_e4m3_codebook_and_saturation():
+    v = O.e4m3_values()
+    assert v[0] == 0 and v[1] == 2.0 ** -9 and v[126] == 448.0 and v[56] == 1.0
+    assert np.all(np.diff(v) > 0)
+    assert O.e4m3_encode(np.array([448.0, 470.0, 1e6], np.float32)).tolist() == [126, 126, 126]
+
+
+def test_fp8_scales_sizes_and_error_bound():
+    rng = np.random.default_rng(52)
+    w = (rng.normal(size=(64, 1024)) * 0.02).astype(np.float32)
+    q = O.nf4_quantize_fp8(w)
+    blocks = w.size // 64
+    assert q["q8"].size == blocks and q["s2"].size == -(-blocks // 256)
+    bits = (8 * blocks + 32 * q["s2"].size) / w.size            # second-level cost per weight
+    assert abs(bits - (0.125 + 32 / 16384)) < 1e-12              # BEA's 0.125 plus the group scales
+    ref = O.nf4_quantize(w, double_quant=False)
+    assert np.array_equal(q["codes"], ref["codes"])             # codes from the fp32 absmax
+    rec = (O.e4m3_values()[q["q8"]] * np.repeat(q["s2"], 256)[:blocks]).astype(np.float32)
+    a = ref["absmax"].astype(np.float64)
+    # E4M3 keeps 3 mantissa bits: <= 2^-4 relative in the normal range (the
+    # group scale puts the largest absmax at 448, so blocks within 2^14 of it
+    # stay normal)
+    normal = a >= a.max() * 2.0 ** -14
+    assert np.all(np.abs(rec[normal] - a[normal]) <= 2.0 ** -4 * a[normal] * (1 + 1e-6))
+
+
+def test_fp8_dequantise_uses_the_reconstructed_absmax():
+    w = np.zeros((4, 512), np.float32)
+    w[1, 70] = 0.5; w[2, 300] = -0.25
+    q = O.nf4_quantize_fp8(w)
+    Wh = O.bf16_to_f32(O.nf4_dequantize_fp8(q))
+    # a block whose absmax is the group maximum reconstructs it exactly
+    # (448 * m / 448 rounds back to m) and its extreme weight is +-absmax
+    assert Wh[1, 70] == 0.5 and Wh[2, 300] == -0.25
+    assert np.all(Wh[0] == 0) and np.all(Wh[3] == 0)
+    z = O.nf4_quantize_fp8(np.zeros((2, 256), np.float32))
+    assert np.all(z["s2"] == 0) and np.all(z["q8"] == 0)
