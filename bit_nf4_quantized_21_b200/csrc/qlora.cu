@@ -828,17 +828,52 @@ namespace {
 
 __device__ __align__(256) uint8_t g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
 
+// The address is cached per device together with the id of the context it
+// was looked up in: after a cudaDeviceReset the device's next primary
+// context loads the module afresh and the array may sit elsewhere, so a
+// changed context id triggers a new lookup.  Without the driver's context-id
+// query the address is looked up on every call.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+bool current_ctx_id(unsigned long long* id) {
+  static std::once_flag once;
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_cur || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[64] = {};
+unsigned long long g_noalloc_ctx[64] = {};
 
 qlora_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  unsigned long long ctx = 0;
+  const bool have_id = current_ctx_id(&ctx);
+  if (!have_id || !g_noalloc_ptr[dev] || g_noalloc_ctx[dev] != ctx) {
+    // the lookup also makes the device's primary context current when no
+    // runtime call has done so yet; the context id is read after it
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QLORA_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = current_ctx_id(&ctx) ? ctx : 0;
   }
   *out = g_noalloc_ptr[dev];
   return QLORA_OK;

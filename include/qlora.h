@@ -280,7 +280,11 @@ qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16
  * computes, with the same kernels.
  *
  * Scratch: one file-scope device array of QLORA_NOALLOC_SCRATCH_BYTES
- * (16 MiB) per GPU, held from library load until process exit.  A problem
+ * (16 MiB) per GPU.  CUDA materialises it when the library's device code is
+ * loaded on that GPU -- with lazy module loading (CUDA's default) that is
+ * the first call that runs a kernel of this library there, which therefore
+ * also pays the load; make a warm-up call where that latency matters -- and
+ * it stays until process exit.  A problem
  * whose forward scratch (split-K partials of T, fp32 T, the two bf16 planes
  * of s*T, a padded copy of B when r % 8 != 0) does not fit is rejected with
  * QLORA_ERR_SCRATCH_LIMIT before anything is enqueued; e.g. M = 8192,
@@ -292,7 +296,10 @@ qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16
  * the GPU (different streams, or different host threads) race and give
  * wrong results; serialise them (same stream, or events).  The first call
  * on each device looks up the array's device address with that device
- * current; make that first call before any stream capture.  The call itself
+ * current; make that first call before any stream capture.  The address is
+ * looked up again whenever the device's current context has changed (e.g.
+ * after cudaDeviceReset), so a call after a reset uses the new context's
+ * array; work enqueued before the reset is lost with its context.  The call itself
  * allocates nothing (no cudaMalloc, no cudaFree, no allocating library
  * routine).  Arguments as for qlora_linear_fwd, minus the workspace.
  */

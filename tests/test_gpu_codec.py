@@ -118,3 +118,44 @@ def test_repeated_calls_are_deterministic():
     b, bh, _ = _roundtrip(W)
     assert torch.equal(a.codes, b.codes) and torch.equal(a.absmax_q8, b.absmax_q8)
     assert torch.equal(ah.view(torch.int16), bh.view(torch.int16))
+
+
+def _sweep_blocks(absmax: float, centres, half_width: int) -> np.ndarray:
+    """fp32 blocks [n, 64]: element 0 is +/-absmax (alternating), elements
+    1..63 walk every binary32 w within `half_width` ulps of fp32(x0 * absmax)
+    for each centre x0, so that the normalised value x = w * fp32(1/absmax)
+    steps across x0 one binary32 at a time (exactly so for absmax a power of
+    two).  Values with |w| > absmax are dropped."""
+    a = np.float32(absmax)
+    vals = []
+    for x0 in centres:
+        w0 = np.float32(np.float64(x0) * np.float64(a))
+        k = np.arange(-half_width, half_width + 1, dtype=np.int64)
+        if w0 == 0:   # the edge at x = 0: the smallest magnitudes of both signs
+            mag = np.arange(1, half_width + 1, dtype=np.int32).view(np.float32)
+            vals.append(np.concatenate([mag, -mag]))
+            continue
+        base = np.int64(np.abs(w0).view(np.int32))
+        mag = (base + k).astype(np.int32).view(np.float32)
+        w = np.where(w0 < 0, -mag, mag).astype(np.float32)
+        vals.append(w[np.abs(w) <= a])
+    v = np.concatenate(vals)
+    nb = -(-v.size // 63)
+    v = np.concatenate([v, np.zeros(nb * 63 - v.size, np.float32)]).reshape(nb, 63)
+    head = np.where(np.arange(nb) % 2 == 0, a, -a).astype(np.float32)[:, None]
+    return np.concatenate([head, v], axis=1)
+
+
+def test_encoder_cells_and_thresholds_swept_binary32():
+    # The kernel counts #{i : x > t_i} through a table of 66 cells of width
+    # 1/32 (one compare per cell).  Sweep every binary32 within 1500 ulps of
+    # each of the 15 thresholds and each of the 65 cell edges j/32, at
+    # absmax values that are powers of two (x = w / absmax exactly) and not,
+    # and require the codes, scales and dequantised weights bit for bit.
+    lv = O.nf4_levels().astype(np.float64)
+    thr = (lv[:-1] + lv[1:]) / 2
+    centres = np.concatenate([thr, np.arange(-32, 33) / 32.0])
+    for absmax in (1.0, 2.0 ** -6, 2.0 ** 5, 0.02, 3.7, 0.0513):
+        W = torch.from_numpy(_sweep_blocks(absmax, centres, 1500))
+        _check_exact(W, dq=True)
+        _check_exact(W, dq=False)

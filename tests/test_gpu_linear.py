@@ -33,10 +33,15 @@ def _run(W, X, dY, A, B, alpha, grad_dtype=torch.float32, save_T=True, want_dX=T
     M, r = X.shape[0], A.shape[0]
     Wq = q.qlora_quantize_nf4(W.to(DEV))
     Xd, dYd, Ad, Bd = (t.to(DEV) for t in (X, dY, A, B))
-    T = torch.full((M, r), float("nan"), dtype=torch.float32, device=DEV) if save_T else None
+    N, K = W.shape
+    nan = lambda shape, dt: torch.full(shape, float("nan"), dtype=dt, device=DEV)
+    # every output starts as NaN: an element a kernel fails to write shows up
+    T = nan((M, r), torch.float32) if save_T else None
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
-    Y = q.qlora_linear_fwd(Xd, Wq, Ad, Bd, alpha, T_save=T, d_status=st)
+    Y = q.qlora_linear_fwd(Xd, Wq, Ad, Bd, alpha, Y=nan((M, N), torch.bfloat16), T_save=T, d_status=st)
     dX, dA, dB = q.qlora_linear_bwd(dYd, Xd, Wq, Ad, Bd, alpha, T_saved=T, grad_dtype=grad_dtype,
+                                    dX=nan((M, K), torch.bfloat16) if want_dX else None,
+                                    dA=nan((r, K), grad_dtype), dB=nan((N, r), grad_dtype),
                                     want_dX=want_dX, d_status=st)
     Wh = q.qlora_dequantize(Wq)
     torch.cuda.synchronize()
@@ -59,7 +64,9 @@ def _compare(got, want, grad_tol=TOL, check_dX=True):
     for k in ("Y", "dX", "dA", "dB") + (("T",) if got["T"] is not None else ()):
         if k == "dX" and not check_dX:
             continue
-        errs[k] = O.rel_fro(f64(got[k]), want[k])
+        g = f64(got[k])
+        assert np.isfinite(g).all(), f"{k}: {int((~np.isfinite(g)).sum())} elements not written"
+        errs[k] = O.rel_fro(g, want[k])
     for k, e in errs.items():
         bar = {"T": 1e-4, "dA": grad_tol, "dB": grad_tol}.get(k, TOL)
         assert e <= bar, f"{k}: relative Frobenius error {e:.3e} > {bar:.1e} (all: {errs})"

@@ -65,7 +65,8 @@ def test_outlier_block_matches_page():
 
 @pytest.mark.parametrize("bits", [4, 8])
 def test_int_grid_error_at_most_half_step(bits):
-    # "the gap w - w^ is quantization error, at worst half a grid step"
+    # "QLoRA" (learning-llms page), the paragraph after the absmax equation:
+    # rounding to the grid moves each weight by no more than half a step
     for seed in range(10):
         w = inputs.normal((64,), 1.0, seed, dtype=torch.float32).numpy()
         q, scale, w_hat = O.absmax_int_quantize(w, bits=bits)
@@ -89,7 +90,7 @@ def test_int4_widget_statistics_and_spread():
     # statistical consistency with the widget's sample (its values are not printed)
     assert abs(np.mean(means) - float(kv["mean_abs_error"][0])) < 0.012
     assert abs(np.mean(worsts) - float(kv["worst_error"][0])) < 0.03
-    # "~18x wider": the step ratio is 127/7 exactly; measured mean-error ratio near it
+    # the page puts the int4 error spread at about 18x the int8 one: the step ratio is 127/7 exactly; measured mean-error ratio near it
     assert round(127 / 7) == int(float(kv["int4_vs_int8_spread"][0]))
     assert abs(np.mean(ratios) - 127 / 7) < 1.5
 
