@@ -607,6 +607,55 @@ def config_workloads(q, dev, hbm):
     return out
 
 
+def paged_adam(q, master, mom1, mom2, grad, pbf, status, l2buf, hbm):
+    """The Adam step over paged optimiser state (CUDA managed memory from
+    qlora_paged_alloc), the same n parameters as adam_step: with the state
+    resident on the GPU; paged out to the host before each step, which
+    faults it back in; and paged out, then prefetched back inside the timed
+    region.  Migration bytes per step in the last two: 12 B per parameter."""
+    import ctypes
+    import numpy as np
+    n = master.numel()
+    stream = torch.cuda.current_stream()
+    ptrs = [q.qlora_paged_alloc(4 * n) for _ in range(3)]
+    try:
+        for ptr, src in zip(ptrs, (master, mom1, mom2)):
+            np.ctypeslib.as_array((ctypes.c_float * n).from_address(ptr))[:] = src.cpu().numpy()
+        step_no = [0]
+
+        def step():
+            step_no[0] += 1
+            rc = q.lib().qlora_adam_step(ptrs[0], ptrs[1], ptrs[2], pbf.data_ptr(), grad.data_ptr(), 0, n,
+                                         step_no[0], 1e-4, 0.9, 0.999, 1e-8, 0.01, 1.0, status.data_ptr(),
+                                         stream.cuda_stream)
+            assert rc == 0
+
+        def page(to_device):
+            for ptr in ptrs:
+                q.qlora_paged_prefetch(ptr, 4 * n, to_device=to_device, stream=stream)
+
+        res = {}
+        page(True)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            step()
+        res["resident_us"] = statistics.median(time_events(step, 10, flush=lambda: l2buf.add_(1))) * 1e3
+        res["paged_out_fault_in_us"] = statistics.median(
+            time_events(step, 5, flush=lambda: (page(False), torch.cuda.synchronize()))) * 1e3
+        res["paged_out_prefetch_back_us"] = statistics.median(
+            time_events(lambda: (page(True), step()), 5, flush=lambda: (page(False), torch.cuda.synchronize()))) * 1e3
+        torch.cuda.synchronize()
+        assert status.item() == 0, f"device status {status.item()}"
+    finally:
+        torch.cuda.synchronize()
+        for ptr in ptrs:
+            q.qlora_paged_free(ptr)
+    return {"unit": "us per step", "params": n, **{k: round(v, 2) for k, v in res.items()},
+            "resident_gbs": round(30 * n / (res["resident_us"] * 1e-6) / 1e9, 1),
+            "resident_frac_of_hbm": round(30 * n / (res["resident_us"] * 1e-6) / 1e9 / hbm, 4),
+            "state": "fp32 master, m, v in CUDA managed memory (qlora_paged_alloc); grad and bf16 copy in device memory"}
+
+
 def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_params):
     hbm = float(peaks["hbm_gbs"])
     out = {}
@@ -682,6 +731,7 @@ def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_param
                         "us": round(ms * 1e3, 2), "frac_of_hbm": round(agbs / hbm, 4),
                         "workload": "Adam over the adapters of the 32-layer 7B stack (r = 16)"}
     assert layer.status.item() == 0, f"device status {layer.status.item()}"
+    out["adam_step_paged"] = paged_adam(q, master, mom1, mom2, grad, pbf, layer.status, l2buf, hbm)
     del master, mom1, mom2, grad, pbf
     torch.cuda.empty_cache()
     # decode-shaped forward: 70B MLP weights, M in {1, 4, 16}

@@ -49,6 +49,15 @@ __device__ __forceinline__ uint32_t nf4_encode(float x, const uint2* s_cell) {
   return e.y + ((x > __uint_as_float(e.x)) ? 1u : 0u);
 }
 
+// E4M3 code of a non-negative float: round to nearest even, values above
+// 448 saturate to 448 (the hardware conversion of two floats packs the
+// second operand into the low byte).
+__device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return static_cast<uint32_t>(r) & 0xFFu;
+}
+
 // K1.  Grid: one CTA per group of 256 blocks (16384 weights).  Eight threads
 // share a 64-weight block (8 weights each, one 16-byte load of bf16), so a
 // warp reads 4 whole blocks = 512 contiguous bytes and writes 128 contiguous
@@ -127,10 +136,17 @@ __global__ void __launch_bounds__(kQuantThreads, sizeof(T) == 2 ? 5 : 3)
   m = s_wmax[0];
 #pragma unroll
   for (int i = 1; i < kQuantThreads / 32; ++i) m = fmaxf(m, s_wmax[i]);
-  const float step = (m >= FLT_MIN) ? __fdiv_rn(m, 255.0f) : 0.0f;
+  // linear 8-bit: s2 = m / 255, q = min(255, rint(absmax / s2));
+  // FP8 E4M3: s2 = m / 448 (E4M3's largest finite value), q = E4M3 code of
+  // absmax / s2, round to nearest even, saturating
+  const bool fp8 = dq == kDqE4M3;
+  const float step = (m >= FLT_MIN) ? __fdiv_rn(m, fp8 ? 448.0f : 255.0f) : 0.0f;
   if (tid < nb) {
-    float q = 0.0f;
-    if (step > 0.0f) q = fminf(rintf(__fdiv_rn(a, step)), 255.0f);
+    uint32_t q = 0;
+    if (step > 0.0f) {
+      const float v = __fdiv_rn(a, step);
+      q = fp8 ? f32_to_e4m3(v) : static_cast<uint32_t>(fminf(rintf(v), 255.0f));
+    }
     q8[b0 + tid] = static_cast<uint8_t>(q);
   }
   if (tid == 0) s2[g] = step;
@@ -154,11 +170,12 @@ __global__ void __launch_bounds__(kDeqThreads)
     const uint4* cp = reinterpret_cast<const uint4*>(codes + b * 32);
     const uint4 c0 = __ldg(cp), c1 = __ldg(cp + 1);
     const NF4Table t = nf4_table(nf4_block_scale(q8, s2, absmax_f32, dq, b));
+    const NF4Shr sh = nf4_shr();
     const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       uint32_t o[4];
-      nf4_decode8(cw[c], t, o);
+      nf4_decode8(cw[c], t, o, sh);
       stage[warp][lane * 8 + (c ^ (lane & 7))] = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }

@@ -58,11 +58,39 @@ struct GemmArgs {
   int64_t out_cols;      // N (fwd) or K (dX)
   int64_t ldo;           // leading dimension of out
   __nv_bfloat16* out;
+  float* out_f32;        // when non-null, the output goes here in fp32 instead (unrounded)
   int num_kt;            // contraction stages over the weight
   int lora_r16;          // adapter rank rounded up to 16 (0: no adapter)
   int64_t lora_lo_row;   // row of the adapter operand where the lo plane starts (= M)
   int* status;
 };
+
+// Output columns [gc, gc + 16) of row `row` (fp32 accumulator words r):
+// rounded once to bf16 into args.out, or kept fp32 in args.out_f32.
+__device__ __forceinline__ void gemm_store16(const GemmArgs& args, int64_t row, int64_t gc, const uint32_t (&r)[16]) {
+  const bool whole = gc + 16 <= args.out_cols;
+  if (args.out_f32) {
+    float* dst = args.out_f32 + row * args.ldo + gc;
+    if (whole && (args.ldo & 3) == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(dst)[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+    } else {
+      for (int i = 0; i < 16 && gc + i < args.out_cols; ++i) dst[i] = __uint_as_float(r[i]);
+    }
+    return;
+  }
+  uint32_t pk[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+  __nv_bfloat16* dst = args.out + row * args.ldo + gc;
+  if (whole && (args.ldo & 7) == 0) {
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  } else {
+    const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(pk);
+    for (int i = 0; i < 16 && gc + i < args.out_cols; ++i) dst[i] = hv[i];
+  }
+}
 
 struct GemmSmem {
   uint8_t* base;  // 1024-aligned
@@ -158,7 +186,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int it = max(0, issued - kGemmStages); it < issued; ++it) {
           const uint32_t fa = smem_u32(&full_a[it % kGemmStages]);
           const uint64_t t0 = global_ns();
-          while (!mbar_try_wait(fa, (it / kGemmStages) & 1) && global_ns() - t0 < 200000000ull) {}
+          while (!mbar_try_wait(fa, (it / kGemmStages) & 1) && global_ns() - t0 < qlora_drain_limit()) {}
         }
       }
     }
@@ -231,11 +259,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             c1 = *reinterpret_cast<const uint4*>(sm.c(s) + row_base + (((ch + 1) ^ cswz) << 4));
           }
           const NF4Table tab = nf4_table(scale);
+          const NF4Shr sh = nf4_shr();
           const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t o[4];
-            nf4_decode8(cw[c], tab, o);
+            nf4_decode8(cw[c], tab, o, sh);
             *reinterpret_cast<uint4*>(wdst + ((static_cast<uint32_t>(c) ^ wswz) << 4)) =
                 make_uint4(o[0], o[1], o[2], o[3]);
           }
@@ -257,10 +286,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     {
       // bounded wait that ignores the abort flag: MMAs may still be running
       const uint32_t bar = smem_u32(acc_full);
-      const uint64_t t0 = global_ns();
+      const uint64_t t0 = global_ns(), limit = qlora_wait_limit();
       bool ok = true;
       while (!mbar_try_wait(bar, 0)) {
-        if (global_ns() - t0 > QLORA_WAIT_NS) { ok = false; break; }
+        if (global_ns() - t0 > limit) { ok = false; break; }
       }
       if (!ok) {
         *abort_flag = 1;
@@ -280,19 +309,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld16(taddr + col, r);
         tmem_ld_wait();
         const int64_t gc = n0 + col;
-        if (row < args.M && gc < args.out_cols) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-          __nv_bfloat16* dst = args.out + row * args.ldo + gc;
-          if (gc + 16 <= args.out_cols && (args.ldo & 7) == 0) {
-            reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          } else {
-            const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(pk);
-            for (int i = 0; i < 16 && gc + i < args.out_cols; ++i) dst[i] = hv[i];
-          }
-        }
+        if (row < args.M && gc < args.out_cols) gemm_store16(args, row, gc, r);
       }
     }
   }

@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int it = max(0, issued - kPairRingA); it < issued; ++it) {
           const uint32_t fa = smem_u32(&full_a[it % kPairRingA]);
           const uint64_t t1 = global_ns();
-          while (!mbar_try_wait_cluster(fa, par(it, kPairRingA)) && global_ns() - t1 < 200000000ull) {}
+          while (!mbar_try_wait_cluster(fa, par(it, kPairRingA)) && global_ns() - t1 < qlora_drain_limit()) {}
         }
       }
     }
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int it = max(0, issued - kPairRingC); it < issued; ++it) {
           const uint32_t fc = smem_u32(&full_c[it % kPairRingC]);
           const uint64_t t0 = global_ns();
-          while (!mbar_try_wait(fc, par(it, kPairRingC)) && global_ns() - t0 < 200000000ull) {}
+          while (!mbar_try_wait(fc, par(it, kPairRingC)) && global_ns() - t0 < qlora_drain_limit()) {}
         }
       }
     }
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     bool live = g >= total || fetch(g, n0, n1);
     for (int it = g; it < total && live; it += G) {
       const int ic = it % kPairRingC, iw = it % kPairRingW;
-      const float scale = args.dq ? __fmul_rn(static_cast<float>(q0), s0) : s0;
+      const float scale = args.dq ? __fmul_rn(dq_value(q0, args.dq), s0) : s0;
       const uint4 c0 = n0, c1 = n1;
       const int64_t n = wn0 + wn_step * it, k = kb0 + kb_step * it;
       const bool valid = it < args.num_kt && n < args.wN && k < KB;
@@ -310,11 +310,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         uint8_t* wdst = slot_w(it) + w_off;
         if (valid) {
           const NF4Table tab = nf4_table(scale);
+          const NF4Shr sh = nf4_shr();
           const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t o[4];
-            nf4_decode8(cw[c], tab, o);
+            nf4_decode8(cw[c], tab, o, sh);
             *reinterpret_cast<uint4*>(wdst + ((static_cast<uint32_t>(c) ^ w_swz) << 4)) =
                 make_uint4(o[0], o[1], o[2], o[3]);
           }
@@ -346,10 +347,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     // ------------------------------------------------------------ epilogue
     {
       const uint32_t bar = smem_u32(acc_full);
-      const uint64_t t0 = global_ns();
+      const uint64_t t0 = global_ns(), limit = qlora_wait_limit();
       bool ok = true;
       while (!mbar_try_wait_cluster(bar, 0)) {
-        if (global_ns() - t0 > QLORA_WAIT_NS) { ok = false; break; }
+        if (global_ns() - t0 > limit) { ok = false; break; }
       }
       if (!ok) {
         *abort_flag = 1;
@@ -371,19 +372,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r1[i]));
         const int64_t gc = np0 + col;
-        if (row < args.M && gc < args.out_cols) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-          __nv_bfloat16* dst = args.out + row * args.ldo + gc;
-          if (gc + 16 <= args.out_cols && (args.ldo & 7) == 0) {
-            reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          } else {
-            const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(pk);
-            for (int i = 0; i < 16 && gc + i < args.out_cols; ++i) dst[i] = hv[i];
-          }
-        }
+        if (row < args.M && gc < args.out_cols) gemm_store16(args, row, gc, r);
       }
     }
   }

@@ -102,7 +102,8 @@ struct GvArgs {
   int M;                     // tokens (1..16)
   int r;                     // adapter rank
   float s;                   // alpha / r
-  const __nv_bfloat16* X;    // [M, K] activations (row stride K)
+  float tscale;              // T = (X A^T) * tscale (1 / (1 - p) under dropout, else 1)
+  const __nv_bfloat16* X;    // [M, K] the adapter's input for T (the activations, or their dropout)
   const __nv_bfloat16* A;    // [r, K] adapter down-projection
   float* T;                  // [M, r] fp32 out: X A^T (unscaled)
   float* tpart;              // [G][M][r] partials of T
@@ -204,7 +205,7 @@ __device__ __forceinline__ bool gv_grid_arrive_wait(int* ctr, int64_t G, int et,
       asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
       if (v >= G) break;
       if (*abort_flag) { ok = false; break; }
-      if (global_ns() - t0 > QLORA_WAIT_NS) {
+      if (global_ns() - t0 > qlora_wait_limit()) {
         *abort_flag = 1;
         if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
         ok = false;
@@ -238,7 +239,7 @@ __device__ __forceinline__ bool gv_adapter_T(const GvArgs& args, int64_t c, int6
   for (int64_t o = o0 + et; o < o1; o += 128) {
     float t = 0.0f;
     for (int64_t cc = 0; cc < G; ++cc) t += __ldcg(args.tpart + cc * MR + o);
-    args.T[o] = t;
+    args.T[o] = t * args.tscale;
   }
   if (!gv_grid_arrive_wait(args.tcnt + 1, G, et, abort_flag, args.status)) return false;
   for (int i = et; i < MR; i += 128) sT[i] = args.s * __ldcg(args.T + i);
@@ -331,10 +332,10 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         for (int it = max(0, issued - kGvStages); it < issued; ++it) {
           const uint32_t fc = smem_u32(&fullc[it % kGvStages]);
           const uint64_t t0 = global_ns();
-          while (!mbar_try_wait(fc, (it / kGvStages) & 1) && global_ns() - t0 < 200000000ull) {}
+          while (!mbar_try_wait(fc, (it / kGvStages) & 1) && global_ns() - t0 < qlora_drain_limit()) {}
           const uint32_t rb = smem_u32(&ready[it % kGvStages]);
           const uint64_t t1 = global_ns();
-          while (!mbar_try_wait(rb, (it / kGvStages) & 1) && global_ns() - t1 < 200000000ull) {}
+          while (!mbar_try_wait(rb, (it / kGvStages) & 1) && global_ns() - t1 < qlora_drain_limit()) {}
         }
       }
     }
@@ -394,6 +395,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t c_off = row * (kGvKS / 2), c_swz = (row >> 1) & 3;   // 64-byte rows, 64-byte swizzle
     constexpr int GG = kGvGroups;
+    const NF4Shr sh = nf4_shr();
     // raw block-scale inputs (two blocks) of this thread's stages, loaded one
     // own stage ahead; the cursor (pit, pt, pku) walks stages g, g + 3, ...
     int pit = g;
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       const int s = it % kGvStages;
       float scale[2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) scale[h] = args.dq ? __fmul_rn(static_cast<float>(qa[h]), sa[h]) : sa[h];
+      for (int h = 0; h < 2; ++h) scale[h] = args.dq ? __fmul_rn(dq_value(qa[h], args.dq), sa[h]) : sa[h];
 #pragma unroll
       for (int h = 0; h < 2; ++h) { qa[h] = qb[h]; sa[h] = sb[h]; }
       load_next(qb, sb);
@@ -452,7 +454,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
           uint32_t d[4];
-          nf4_decode8(cw[w], tab, d);
+          nf4_decode8(cw[w], tab, d, sh);
           o[4 * w + 0] = d[0]; o[4 * w + 1] = d[1]; o[4 * w + 2] = d[2]; o[4 * w + 3] = d[3];
         }
         tmem_st32(tcol + 32u * h, o);
@@ -586,7 +588,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       const uint64_t t0 = global_ns();
       while (!mbar_try_wait(bars2[i], 0)) {
         __nanosleep(64);
-        if (global_ns() - t0 > QLORA_WAIT_NS) {
+        if (global_ns() - t0 > qlora_wait_limit()) {
           *abort_flag = 1;
           if (args.status) atomicOr(args.status, QLORA_DEV_TIMEOUT);
           break;

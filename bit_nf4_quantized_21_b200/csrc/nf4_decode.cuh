@@ -40,17 +40,29 @@ __device__ __forceinline__ NF4Table nf4_table(float scale) {
   return t;
 }
 
+// The decode's three right shifts are done as high halves of multiplies
+// (x >> k == mulhi(x, 2^(32 - k))): a multiply issues on the FMA pipe, while
+// every byte permute and mask of the lookup issues on the integer pipe, which
+// is the decode's bottleneck.  The multipliers are read from constant memory
+// so that the compiler cannot turn the multiplies back into shifts.
+__constant__ uint32_t c_nf4_shr[2] = {0x80000000u /* >> 1 */, 0x00010000u /* >> 16 */};
+struct NF4Shr {
+  uint32_t m1, m16;
+};
+__device__ __forceinline__ NF4Shr nf4_shr() { return NF4Shr{c_nf4_shr[0], c_nf4_shr[1]}; }
+
 // 8 codes (one 32-bit word; code i in bits 4i..4i+3) -> 8 bf16 in 4 words,
 // element 2j in the low half of word j.
-__device__ __forceinline__ void nf4_decode8(uint32_t w, const NF4Table& t, uint32_t (&o)[4]) {
-  const uint32_t idx = w & 0x77777777u;                              // low 3 bits of every code
-  const uint32_t half = ((w >> 1) & 0x44444444u) | 0x32103210u;      // byte i from word A or B
+__device__ __forceinline__ void nf4_decode8(uint32_t w, const NF4Table& t, uint32_t (&o)[4],
+                                            NF4Shr sh = NF4Shr{0x80000000u, 0x00010000u}) {
+  const uint32_t idx = w & 0x77777777u;                                      // low 3 bits of every code
+  const uint32_t half = (__umulhi(w, sh.m1) & 0x44444444u) | 0x32103210u;    // byte i from word A or B
   // prmt reads only the low 16 bits (four nibbles) of its selector, so the
   // upper half of idx / half needs no masking for h = 0
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint32_t s = h ? (idx >> 16) : idx;
-    const uint32_t g = h ? (half >> 16) : half;
+    const uint32_t s = h ? __umulhi(idx, sh.m16) : idx;
+    const uint32_t g = h ? __umulhi(half, sh.m16) : half;
     const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], s), prmt(t.lo[2], t.lo[3], s), g);
     const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], s), prmt(t.hi[2], t.hi[3], s), g);
     o[2 * h] = prmt(lo, hi, 0x5140u);
@@ -58,12 +70,31 @@ __device__ __forceinline__ void nf4_decode8(uint32_t w, const NF4Table& t, uint3
   }
 }
 
+// Second-level scale formats (the weight's double_quant field): none (fp32
+// block absmax), linear 8-bit (q * s2), and FP8 E4M3 codes (E4M3(q) * s2,
+// "QLoRA", infra.bea.ai, §1 subsection "Double Quantization", which
+// quantises the block scales to FP8).
+constexpr int kDqNone = 0, kDqU8 = 1, kDqE4M3 = 2;
+
+// Value of an E4M3 code 0..126 (bias 7, 3 mantissa bits; no sign, no NaN:
+// the quantiser writes only non-negative finite codes): the exponent field
+// moves to fp32's bias, the 3 mantissa bits to the top of fp32's mantissa;
+// exponent field 0 is the subnormal range m * 2^-9.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+  const uint32_t e = c >> 3, m = c & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0x1p-9f;
+}
+// The stored 8-bit value of a block's absmax as a float.
+__device__ __forceinline__ float dq_value(uint32_t q, int dq) {
+  return dq == kDqE4M3 ? e4m3_to_f32(q) : static_cast<float>(q);
+}
+
 // Block scale of the stored format.
 __device__ __forceinline__ float nf4_block_scale(const uint8_t* __restrict__ q8,
                                                  const float* __restrict__ s2,
                                                  const float* __restrict__ absmax_f32, int dq,
                                                  int64_t b) {
-  if (dq) return __fmul_rn(static_cast<float>(__ldg(q8 + b)), __ldg(s2 + (b >> 8)));
+  if (dq) return __fmul_rn(dq_value(__ldg(q8 + b), dq), __ldg(s2 + (b >> 8)));
   return __ldg(absmax_f32 + b);
 }
 

@@ -2,7 +2,8 @@
 // loads, tcgen05 (TMEM allocation, MMA, commit, loads) and the shared-memory
 // matrix descriptors the tensor cores read.
 //
-// Every mbarrier wait here is bounded: after QLORA_WAIT_NS of global time it
+// Every mbarrier wait here is bounded: after a fixed time (QLORA_WAIT_NS, 2 s by
+// default; see qlora_wait_limit) it
 // records a timeout bit in the caller's status word (if any), raises the
 // CTA-local abort flag, and returns false so that the role can wind down
 // instead of spinning forever.
@@ -21,6 +22,19 @@
 #define QLORA_DEV_TIMEOUT 2
 
 namespace qlora {
+
+// The wait bound in ns of global time: QLORA_WAIT_NS unless a test shortens
+// it for the device (qlora_debug_set_wait_limit); read only once a wait has
+// gone on for a while.  Abort-path drains of copies in flight use the same
+// bound, capped at 200 ms.
+__device__ unsigned long long g_qlora_wait_ns = QLORA_WAIT_NS;
+__device__ __forceinline__ uint64_t qlora_wait_limit() {
+  return *reinterpret_cast<volatile unsigned long long*>(&g_qlora_wait_ns);
+}
+__device__ __forceinline__ uint64_t qlora_drain_limit() {
+  const uint64_t w = qlora_wait_limit();
+  return w < 200000000ull ? w : 200000000ull;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -58,6 +72,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test: unlike try_wait, which may suspend the thread for a
+// while when the phase is incomplete, test_wait returns at once -- for a
+// thread that polls several barriers and must not stall on any one.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait.  `abort_flag` is a CTA-shared word: once any role has given
 // up, the others stop waiting too.  Returns false on timeout/abort.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
@@ -69,7 +98,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > QLORA_WAIT_NS) {
+      if (global_ns() - t0 > qlora_wait_limit()) {
         *abort_flag = 1;
         if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
         return false;
@@ -90,7 +119,7 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, v
     __nanosleep(ns);
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_ns() - t0 > QLORA_WAIT_NS) {
+    if (global_ns() - t0 > qlora_wait_limit()) {
       *abort_flag = 1;
       if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
       return false;
@@ -258,7 +287,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > QLORA_WAIT_NS) {
+      if (global_ns() - t0 > qlora_wait_limit()) {
         *abort_flag = 1;
         if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
         return false;

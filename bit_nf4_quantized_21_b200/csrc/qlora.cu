@@ -27,6 +27,7 @@
 #include "gemv_nf4.cuh"
 #include "adam.cuh"
 #include "merge.cuh"
+#include "dropout.cuh"
 
 using namespace qlora;
 
@@ -121,7 +122,7 @@ qlora_status check_weight(const qlora_nf4_weight* w, bool need_arrays) {
   if (w->rows < 1 || w->cols < 64 || (w->cols % 64) != 0) return QLORA_ERR_INVALID_ARG;
   if (w->rows > (int64_t(1) << 31) || w->cols > (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
   if (w->blocksize != 64 || w->group != 256) return QLORA_ERR_UNSUPPORTED;
-  if (w->reserved != 0 || (w->double_quant != 0 && w->double_quant != 1)) return QLORA_ERR_INVALID_ARG;
+  if (w->reserved != 0 || w->double_quant < kDqNone || w->double_quant > kDqE4M3) return QLORA_ERR_INVALID_ARG;
   if (!need_arrays) return QLORA_OK;
   if (!w->codes || !aligned16(w->codes)) return QLORA_ERR_INVALID_ARG;
   if (w->double_quant) {
@@ -185,6 +186,7 @@ struct SkJob {
 
 SkinnyArgs sk_args(const SkPlan& pl, float* partial, unsigned int* cnt, int* status) {
   SkinnyArgs a{};
+  a.vscale = 1.0f;
   a.P = pl.P;
   a.Qn = pl.Qn;
   a.Qtot = pl.Qtot;
@@ -288,8 +290,48 @@ Ws ws_layout(const Dims& d) {
   return w;
 }
 
+// LoRA dropout of one call: Philox key, the integer cut ceil(p 2^32) and
+// fp32(1 / (1 - p)).
+struct DropCfg {
+  uint64_t seed, thr;
+  float inv_q;
+};
+bool dropout_cfg(double p, uint64_t seed, DropCfg* c) {
+  if (!std::isfinite(p) || p < 0.0 || p >= 1.0) return false;
+  c->seed = seed;
+  c->thr = static_cast<uint64_t>(std::ceil(p * 4294967296.0));
+  c->inv_q = static_cast<float>(1.0 / (1.0 - p));
+  return true;
+}
+// Workspace of the dropout entries: the plain layout, then X * keep (bf16
+// [M, K]), the frozen-path dX in fp32 ([M, K]) and G in fp32 ([M, r]).
+struct WsDrop {
+  size_t xd, dxf, g32, total;
+};
+WsDrop ws_drop_layout(const Dims& d) {
+  auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  WsDrop w{};
+  size_t off = ws_layout(d).total;
+  w.xd = off; off += a256(static_cast<size_t>(d.M) * d.K * 2);
+  w.dxf = off; off += a256(static_cast<size_t>(d.M) * d.K * 4);
+  w.g32 = off; off += a256(static_cast<size_t>(d.M) * d.r * 4);
+  w.total = off;
+  return w;
+}
+unsigned dropout_grid(int64_t items) {
+  const int sms = std::max(1, sm_count());
+  return static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(cdiv(items, kDropThreads), 16LL * sms)));
+}
+// Xd = X * keep over the M x K activations.
+qlora_status run_dropout_x(const void* X, void* Xd, const Dims& d, const DropCfg& c, cudaStream_t cs) {
+  const int64_t n = d.M * d.K;
+  k_dropout_x<<<dropout_grid(n / 8), kDropThreads, 0, cs>>>(static_cast<const __nv_bfloat16*>(X),
+                                                              static_cast<__nv_bfloat16*>(Xd), n, c.seed, c.thr);
+  return check_launch();
+}
+
 qlora_status check_linear(int64_t M, const qlora_nf4_weight* Wq, int r, float alpha, const void* workspace,
-                          size_t ws_bytes) {
+                          size_t ws_bytes, bool dropout = false) {
   qlora_status st = check_weight(Wq, true);
   if (st != QLORA_OK) return st;
   if (M < 1 || M > (int64_t(1) << 31)) return QLORA_ERR_INVALID_ARG;
@@ -297,7 +339,8 @@ qlora_status check_linear(int64_t M, const qlora_nf4_weight* Wq, int r, float al
   if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
   if (Wq->rows % 8 != 0) return QLORA_ERR_UNSUPPORTED;
   if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
-  if (ws_bytes < ws_layout(dims_of(M, Wq->rows, Wq->cols, r)).total) return QLORA_ERR_WORKSPACE;
+  const Dims d = dims_of(M, Wq->rows, Wq->cols, r);
+  if (ws_bytes < (dropout ? ws_drop_layout(d).total : ws_layout(d).total)) return QLORA_ERR_WORKSPACE;
   return QLORA_OK;
 }
 
@@ -321,7 +364,7 @@ qlora_status clear_counters(uint8_t* ws, const Ws& L, const SkPlans& p, cudaStre
 // T = X A^T  (fp32 into t32, and optionally s*T in bf16 planes into sx), one
 // launch.  The caller has cleared the counters.
 qlora_status run_T(const void* X, const void* A, const Dims& d, float s, uint8_t* ws, const Ws& L, float* t32,
-                   __nv_bfloat16* sx, int* status, cudaStream_t st) {
+                   __nv_bfloat16* sx, int* status, cudaStream_t st, float vscale = 1.0f) {
   const SkPlans P = plans_of(d);
   SkJob j;
   j.pl = P.T;
@@ -329,6 +372,7 @@ qlora_status run_T(const void* X, const void* A, const Dims& d, float s, uint8_t
   if (!bf16_map(&j.tb, A, d.K, d.r, d.K, 64, static_cast<uint32_t>(j.pl.Qn))) return QLORA_ERR_CUDA;
   j.a = sk_args(j.pl, reinterpret_cast<float*>(ws + L.partial), cnt_T(ws, L), status);
   sk_rows(j.a, d, s, t32, sx, nullptr);
+  j.a.vscale = vscale;
   return launch_skinny<0, 0>(j, nullptr, st);
 }
 
@@ -370,7 +414,7 @@ qlora_status launch_gemm(int mode, const CUtensorMap& tact, const CUtensorMap& t
 // [N, K] (plain LoRA; always the 2-SM pair kernel).
 qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, const void* Wdense, const Dims& d,
                        const void* la, const void* lb, void* out, const qlora_gemm_events* ev, int* status,
-                       cudaStream_t cs) {
+                       cudaStream_t cs, float* out_f32 = nullptr, bool fold = true) {
   const bool dense = Wdense != nullptr;
   const bool pair = d.M > 128 || dense;
   const bool fwd = mode == kModeFwd;
@@ -408,8 +452,9 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   a.out_cols = fwd ? d.N : d.K;
   a.ldo = a.out_cols;
   a.out = static_cast<__nv_bfloat16*>(out);
+  a.out_f32 = out_f32;
   a.num_kt = static_cast<int>(fwd ? d.K / 64 : cdiv(d.N, 64));
-  a.lora_r16 = d.r16;
+  a.lora_r16 = fold ? d.r16 : 0;
   a.lora_lo_row = d.M;
   a.status = status;
   if (!pair) return launch_gemm(mode, tact, tcodes, tla, tlb, a, ev, cs);
@@ -450,7 +495,8 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
 // the T phases wait across CTAs).  One memset clears the counters first.
 qlora_status run_gemv(const void* X, const void* A, const qlora_nf4_weight* Wq, const Dims& d, float* t32,
                       const void* B, void* Y, float alpha_over_r, uint8_t* ws, const Ws& L,
-                      const qlora_gemm_events* ev, int* status, cudaStream_t cs) {
+                      const qlora_gemm_events* ev, int* status, cudaStream_t cs, const void* Xt = nullptr,
+                      float tscale = 1.0f) {
   if (d.r > kGvMaxRank) return QLORA_ERR_UNSUPPORTED;
   const int64_t tiles = cdiv(d.N, kGvRows);
   const int64_t KU = cdiv(d.K, kGvKS);
@@ -465,8 +511,8 @@ qlora_status run_gemv(const void* X, const void* A, const qlora_nf4_weight* Wq, 
     return QLORA_ERR_CUDA;
   GvArgs a{};
   a.q8 = Wq->absmax_q8; a.s2 = Wq->group_scale; a.absmax_f32 = Wq->absmax_f32; a.dq = Wq->double_quant;
-  a.N = d.N; a.K = d.K; a.M = static_cast<int>(d.M); a.r = d.r; a.s = alpha_over_r;
-  a.X = static_cast<const __nv_bfloat16*>(X);
+  a.N = d.N; a.K = d.K; a.M = static_cast<int>(d.M); a.r = d.r; a.s = alpha_over_r; a.tscale = tscale;
+  a.X = static_cast<const __nv_bfloat16*>(Xt ? Xt : X);
   a.A = static_cast<const __nv_bfloat16*>(A);
   a.T = t32;
   a.tpart = reinterpret_cast<float*>(ws + L.gv_tpart);
@@ -504,7 +550,7 @@ qlora_status run_gemv(const void* X, const void* A, const qlora_nf4_weight* Wq, 
 qlora_status linear_bwd_core(const void* dY, const void* X, const Dims& d, const qlora_nf4_weight* Wq,
                              const void* Wdense, const void* A, const void* B, float alpha, const float* T_saved,
                              void* dX, void* dA, void* dB, qlora_dtype grad_dtype, void* workspace, int* d_status,
-                             const qlora_gemm_events* events, cudaStream_t cs) {
+                             const qlora_gemm_events* events, cudaStream_t cs, const DropCfg* drop = nullptr) {
   qlora_status st = QLORA_OK;
   const Ws L = ws_layout(d);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -518,11 +564,21 @@ qlora_status linear_bwd_core(const void* dY, const void* X, const Dims& d, const
   if (st != QLORA_OK) return st;
   st = clear_counters(ws, L, P, cs);
   if (st != QLORA_OK) return st;
+  // the adapter's input: X, or X * keep under dropout (regenerated from the
+  // call's seed, the same mask as the forward's)
+  const WsDrop WD = drop ? ws_drop_layout(d) : WsDrop{};
+  const void* Xa = X;
+  if (drop) {
+    st = run_dropout_x(X, ws + WD.xd, d, *drop, cs);
+    if (st != QLORA_OK) return st;
+    Xa = ws + WD.xd;
+  }
+  const float inv_q = drop ? drop->inv_q : 1.0f;
   // 0. T recomputed when the forward's was not kept
   const float* t = T_saved;
   if (!t) {
     float* t32 = reinterpret_cast<float*>(ws + L.t32);
-    st = run_T(X, A, d, s, ws, L, t32, nullptr, d_status, cs);
+    st = run_T(Xa, A, d, s, ws, L, t32, nullptr, d_status, cs, inv_q);
     if (st != QLORA_OK) return st;
     t = t32;
   }
@@ -534,16 +590,31 @@ qlora_status linear_bwd_core(const void* dY, const void* X, const Dims& d, const
     if (!bf16_map(&j.ta, dY, d.N, d.M, d.N, 64, kSkBM)) return QLORA_ERR_CUDA;
     if (!bf16_map(&j.tb, Bp, d.r8, d.N, d.r8, 64, 64)) return QLORA_ERR_CUDA;
     j.a = sk_args(j.pl, reinterpret_cast<float*>(ws + L.partial), cnt_G(ws, L, P), d_status);
-    sk_rows(j.a, d, s, nullptr, sG, Ghl);
+    // under dropout the adapter term of dX is masked per element, so it is
+    // added after the GEMM from fp32 G instead of folded into it
+    if (drop)
+      sk_rows(j.a, d, s, reinterpret_cast<float*>(ws + WD.g32), nullptr, Ghl);
+    else
+      sk_rows(j.a, d, s, nullptr, sG, Ghl);
     j.a.side_src = t;
     j.a.side_rows = d.M;
     j.a.side_hl = Thl;
     st = launch_skinny<0, 1>(j, nullptr, cs);
     if (st != QLORA_OK) return st;
   }
-  // 2. dX = dY W^ + (sG) A
-  if (dX) {
+  // 2. dX = dY W^ + (sG) A; under dropout dY W^ in fp32, then one pass
+  //    adding s ((G A) * keep) / (1 - p) and rounding once
+  if (dX && !drop) {
     st = run_fused(kModeDx, dY, Wq, Wdense, d, sG, A, dX, events, d_status, cs);
+    if (st != QLORA_OK) return st;
+  } else if (dX) {
+    float* dxf = reinterpret_cast<float*>(ws + WD.dxf);
+    st = run_fused(kModeDx, dY, Wq, Wdense, d, sG, A, dX, events, d_status, cs, dxf, false);
+    if (st != QLORA_OK) return st;
+    k_dropout_dx<<<dropout_grid(d.M * (d.K / 8)), kDropThreads, 0, cs>>>(
+        dxf, reinterpret_cast<const float*>(ws + WD.g32), static_cast<const __nv_bfloat16*>(A), d.M, d.K, d.r,
+        s * inv_q, drop->seed, drop->thr, static_cast<__nv_bfloat16*>(dX));
+    st = check_launch();
     if (st != QLORA_OK) return st;
   }
   // 3. dA = s G^T X (C[k, q] = sum_m X[m, k] Ghl[m, q]) and dB = s dY^T T
@@ -553,7 +624,7 @@ qlora_status linear_bwd_core(const void* dY, const void* X, const Dims& d, const
     SkJob ja, jb;
     ja.pl = P.dA;
     jb.pl = P.dB;
-    if (!bf16_map(&ja.ta, X, d.K, d.M, d.K, 64, 64)) return QLORA_ERR_CUDA;
+    if (!bf16_map(&ja.ta, Xa, d.K, d.M, d.K, 64, 64)) return QLORA_ERR_CUDA;
     if (!bf16_map(&ja.tb, Ghl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
     if (!bf16_map(&jb.ta, dY, d.N, d.M, d.N, 64, 64)) return QLORA_ERR_CUDA;
     if (!bf16_map(&jb.tb, Thl, d.Qh, d.M, d.Qh, 64, 64)) return QLORA_ERR_CUDA;
@@ -565,6 +636,7 @@ qlora_status linear_bwd_core(const void* dY, const void* X, const Dims& d, const
       a->out_bf16 = out_bf16;
     }
     ja.a.transpose = 1;
+    ja.a.s = s * inv_q;
     ja.a.out = dA;
     jb.a.transpose = 0;
     jb.a.out = dB;
@@ -619,7 +691,7 @@ qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int double_quant, size_
                              size_t* absmax_bytes, size_t* group_bytes) {
   if (!codes_bytes || !absmax_bytes || !group_bytes) return QLORA_ERR_INVALID_ARG;
   if (rows < 1 || cols < 64 || cols % 64 != 0) return QLORA_ERR_INVALID_ARG;
-  if (double_quant != 0 && double_quant != 1) return QLORA_ERR_INVALID_ARG;
+  if (double_quant < kDqNone || double_quant > kDqE4M3) return QLORA_ERR_INVALID_ARG;
   const int64_t blocks = rows * cols / 64;
   *codes_bytes = static_cast<size_t>(rows * cols / 2);
   *absmax_bytes = static_cast<size_t>(double_quant ? blocks : 4 * blocks);
@@ -715,6 +787,77 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
                          events, cs);
 }
 
+size_t qlora_workspace_bytes_dropout(int64_t M, int64_t N, int64_t K, int r) {
+  if (M < 1 || N < 1 || K < 64 || K % 64 != 0 || r < 1 || r > 256) return 0;
+  return ws_drop_layout(dims_of(M, N, K, r)).total;
+}
+
+qlora_status qlora_lora_dropout_mask(int64_t M, int64_t K, double p, uint64_t seed, uint8_t* keep, void* stream) {
+  DropCfg c;
+  if (!dropout_cfg(p, seed, &c)) return QLORA_ERR_INVALID_ARG;
+  if (M < 1 || K < 64 || K % 64 != 0 || M > (int64_t(1) << 31) || K > (int64_t(1) << 31))
+    return QLORA_ERR_INVALID_ARG;
+  if (!keep || !aligned16(keep)) return QLORA_ERR_INVALID_ARG;
+  const int64_t n = M * K;
+  k_dropout_mask<<<dropout_grid(n / 4), kDropThreads, 0, static_cast<cudaStream_t>(stream)>>>(keep, n, c.seed, c.thr);
+  return check_launch();
+}
+
+qlora_status qlora_linear_fwd_dropout(const void* X, int64_t M, const qlora_nf4_weight* Wq, const void* A,
+                                      const void* B, int r, float alpha, double p, uint64_t seed, void* Y,
+                                      float* T_save, void* workspace, size_t ws_bytes, int* d_status,
+                                      const qlora_gemm_events* events, void* stream) {
+  qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes, true);
+  if (st != QLORA_OK) return st;
+  DropCfg drop;
+  if (!dropout_cfg(p, seed, &drop)) return QLORA_ERR_INVALID_ARG;
+  if (!X || !A || !B || !Y || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y))
+    return QLORA_ERR_INVALID_ARG;
+  if (T_save && !aligned16(T_save)) return QLORA_ERR_INVALID_ARG;
+  if (!ensure_smem_attrs()) return QLORA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const Dims d = dims_of(M, Wq->rows, Wq->cols, r);
+  const Ws L = ws_layout(d);
+  const WsDrop WD = ws_drop_layout(d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const float s = alpha / static_cast<float>(r);
+  float* t32 = T_save ? T_save : reinterpret_cast<float*>(ws + L.t32);
+  __nv_bfloat16* sT = reinterpret_cast<__nv_bfloat16*>(ws + L.sx);
+  void* Xd = ws + WD.xd;
+  st = run_dropout_x(X, Xd, d, drop, cs);   // the adapter's input X * keep
+  if (st != QLORA_OK) return st;
+  if (M <= kDecodeMaxM)
+    return run_gemv(X, A, Wq, d, t32, B, Y, s, ws, L, events, d_status, cs, Xd, drop.inv_q);
+  st = clear_counters(ws, L, plans_of(d), cs);
+  if (st != QLORA_OK) return st;
+  st = run_T(Xd, A, d, s, ws, L, t32, sT, d_status, cs, drop.inv_q);
+  if (st != QLORA_OK) return st;
+  const void* Bp = padded_B(B, d, ws, L, cs, &st);
+  if (st != QLORA_OK) return st;
+  // the frozen path sees X undropped
+  return run_fused(kModeFwd, X, Wq, nullptr, d, sT, Bp, Y, events, d_status, cs);
+}
+
+qlora_status qlora_linear_bwd_dropout(const void* dY, const void* X, int64_t M, const qlora_nf4_weight* Wq,
+                                      const void* A, const void* B, int r, float alpha, double p, uint64_t seed,
+                                      const float* T_saved, void* dX, void* dA, void* dB, qlora_dtype grad_dtype,
+                                      void* workspace, size_t ws_bytes, int* d_status,
+                                      const qlora_gemm_events* events, void* stream) {
+  qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes, true);
+  if (st != QLORA_OK) return st;
+  DropCfg drop;
+  if (!dropout_cfg(p, seed, &drop)) return QLORA_ERR_INVALID_ARG;
+  if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(dA) || !aligned16(dB))
+    return QLORA_ERR_INVALID_ARG;
+  if ((dX && !aligned16(dX)) || (T_saved && !aligned16(T_saved))) return QLORA_ERR_INVALID_ARG;
+  if (grad_dtype != QLORA_F32 && grad_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (!ensure_smem_attrs()) return QLORA_ERR_CUDA;
+  const Dims d = dims_of(M, Wq->rows, Wq->cols, r);
+  return linear_bwd_core(dY, X, d, Wq, nullptr, A, B, alpha, T_saved, dX, dA, dB, grad_dtype, workspace, d_status,
+                         events, static_cast<cudaStream_t>(stream), &drop);
+}
+
 qlora_status qlora_lora_linear_fwd(const void* X, int64_t M, const void* W, int64_t N, int64_t K, const void* A,
                                    const void* B, int r, float alpha, void* Y, float* T_save, void* workspace,
                                    size_t ws_bytes, int* d_status, const qlora_gemm_events* events, void* stream) {
@@ -792,6 +935,56 @@ qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
   qlora::k_adam_step<<<grid, qlora::kAdamThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return check_launch();
+}
+
+qlora_status qlora_debug_set_wait_limit(uint64_t ns) {
+  const unsigned long long v = ns ? static_cast<unsigned long long>(ns) : QLORA_WAIT_NS;
+  return cudaMemcpyToSymbol(g_qlora_wait_ns, &v, sizeof(v)) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_debug_inject_stall(int on) {
+  const int v = on ? 1 : 0;
+  return cudaMemcpyToSymbol(g_qlora_inject_stall, &v, sizeof(v)) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_paged_alloc(size_t bytes, void** ptr) {
+  if (!ptr) return QLORA_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  if (bytes == 0) return QLORA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  void* p = nullptr;
+  if (cudaMallocManaged(&p, bytes, cudaMemAttachGlobal) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  // resident on the GPU by preference: pages the driver evicts to the host
+  // under memory pressure, or that the caller prefetches there, migrate back
+  // on the GPU's next access
+  if (cudaMemAdvise(p, bytes, cudaMemAdviseSetPreferredLocation, dev) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(p);
+    return QLORA_ERR_CUDA;
+  }
+  *ptr = p;
+  return QLORA_OK;
+}
+
+qlora_status qlora_paged_free(void* ptr) {
+  if (!ptr) return QLORA_OK;
+  return cudaFree(ptr) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_paged_prefetch(void* ptr, size_t bytes, int to_device, void* stream) {
+  if (!ptr || bytes == 0) return QLORA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  const int dst = to_device ? dev : cudaCpuDeviceId;
+  if (cudaMemPrefetchAsync(ptr, bytes, dst, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
 }
 
 qlora_status qlora_merge_nf4(const qlora_nf4_weight* Wq, const void* A, const void* B, int r, float alpha,

@@ -56,6 +56,7 @@ struct SkinnyArgs {
   // the final transform
   int finish;         // kFinRows or kFinGrad
   float s;
+  float vscale;       // rows: every value is multiplied by this first (1 / (1 - p) under dropout, else 1)
   int r, r8, r16, Qh;
   float* f32;                      // rows
   __nv_bfloat16* s_bf16;           // rows
@@ -108,7 +109,10 @@ __device__ __forceinline__ void sk_st8(__nv_bfloat16* dst, const uint32_t* w, in
 // row, so the outputs go out as 16-byte stores (row offsets are multiples of
 // 16 bytes: r8 and r16 are multiples of 8 and 16, Qh of 64; fp32 T takes
 // the vector path when r % 4 == 0).  Values of columns >= r are zero.
-__device__ __forceinline__ void sk_rows_out(const SkinnyArgs& a, int64_t m, int c0, const float (&v)[16]) {
+__device__ __forceinline__ void sk_rows_out(const SkinnyArgs& a, int64_t m, int c0, const float (&v0)[16]) {
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = v0[i] * a.vscale;
   if (a.f32) {
     float* d = a.f32 + m * a.r + c0;
     if ((a.r & 3) == 0 && c0 + 16 <= a.r) {
@@ -176,6 +180,12 @@ __device__ __forceinline__ void sk_grad_out(const SkinnyArgs& a, int64_t p, int 
   }
 }
 
+// Test hook (qlora_debug_inject_stall): when set, CTA 0 of the first problem
+// of every adapter-product launch withholds the loads of its first stage, so
+// that its MMA thread's bounded wait runs out and the launch takes its
+// timeout path (status bit, early exit, TMEM released).
+__device__ int g_qlora_inject_stall = 0;
+
 template <int A_MN, int B_MN>
 __global__ void __launch_bounds__(kSkThreads, 1)
     k_skinny(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
@@ -236,9 +246,14 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       int issued = 0;
+      const bool stall = bid == 0 && !second && *reinterpret_cast<volatile int*>(&g_qlora_inject_stall) != 0;
       for (int it = 0; it < nch; ++it) {
         const int s = it % S;
         if (it >= S && !mbar_wait(smem_u32(&empty[s]), ((it / S) + 1) & 1, abort_flag, args.status)) break;
+        if (stall && it == 0) {   // test hook: this stage's loads are withheld
+          ++issued;
+          continue;
+        }
         const uint32_t fb = smem_u32(&full[s]);
         const uint32_t a_dst = smem_u32(base + s * stage_bytes);
         const uint32_t b_dst = a_dst + kSkABytes;
@@ -261,7 +276,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         for (int it = max(0, issued - S); it < issued; ++it) {
           const uint32_t fb = smem_u32(&full[it % S]);
           const uint64_t t0 = global_ns();
-          while (!mbar_try_wait(fb, (it / S) & 1) && global_ns() - t0 < 200000000ull) {}
+          while (!mbar_try_wait(fb, (it / S) & 1) && global_ns() - t0 < qlora_drain_limit()) {}
         }
       }
     }
@@ -287,10 +302,10 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   } else {
     {
       const uint32_t bar = smem_u32(acc_full);
-      const uint64_t t0 = global_ns();
+      const uint64_t t0 = global_ns(), limit = qlora_wait_limit();
       bool ok = true;
       while (!mbar_try_wait(bar, 0)) {
-        if (global_ns() - t0 > QLORA_WAIT_NS) { ok = false; break; }
+        if (global_ns() - t0 > limit) { ok = false; break; }
       }
       if (!ok) {
         *abort_flag = 1;

@@ -28,7 +28,9 @@ EXPORTED = (
     "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
     "qlora_version", "qlora_linear_fwd_noalloc", "qlora_lora_linear_fwd", "qlora_lora_linear_bwd",
-    "qlora_adam_step", "qlora_merge_nf4",
+    "qlora_adam_step", "qlora_merge_nf4", "qlora_workspace_bytes_dropout", "qlora_lora_dropout_mask",
+    "qlora_linear_fwd_dropout", "qlora_linear_bwd_dropout", "qlora_paged_alloc", "qlora_paged_free",
+    "qlora_paged_prefetch", "qlora_debug_set_wait_limit", "qlora_debug_inject_stall",
 )
 
 
@@ -107,6 +109,27 @@ def lib() -> ctypes.CDLL:
             L.qlora_merge_nf4.argtypes = [ctypes.POINTER(NF4WeightC), P, P, I32, F, P, ctypes.POINTER(NF4WeightC),
                                           P, P]
             L.qlora_merge_nf4.restype = I32
+            D, U64 = ctypes.c_double, ctypes.c_uint64
+            L.qlora_workspace_bytes_dropout.argtypes = [I64, I64, I64, I32]
+            L.qlora_workspace_bytes_dropout.restype = ctypes.c_size_t
+            L.qlora_lora_dropout_mask.argtypes = [I64, I64, D, U64, P, P]
+            L.qlora_lora_dropout_mask.restype = I32
+            L.qlora_linear_fwd_dropout.argtypes = [P, I64, ctypes.POINTER(NF4WeightC), P, P, I32, F, D, U64, P, P,
+                                                   P, ctypes.c_size_t, P, P, P]
+            L.qlora_linear_fwd_dropout.restype = I32
+            L.qlora_linear_bwd_dropout.argtypes = [P, P, I64, ctypes.POINTER(NF4WeightC), P, P, I32, F, D, U64, P,
+                                                   P, P, P, I32, P, ctypes.c_size_t, P, P, P]
+            L.qlora_linear_bwd_dropout.restype = I32
+            L.qlora_paged_alloc.argtypes = [ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]
+            L.qlora_paged_alloc.restype = I32
+            L.qlora_paged_free.argtypes = [P]
+            L.qlora_paged_free.restype = I32
+            L.qlora_paged_prefetch.argtypes = [P, ctypes.c_size_t, I32, P]
+            L.qlora_paged_prefetch.restype = I32
+            L.qlora_debug_set_wait_limit.argtypes = [U64]
+            L.qlora_debug_set_wait_limit.restype = I32
+            L.qlora_debug_inject_stall.argtypes = [I32]
+            L.qlora_debug_inject_stall.restype = I32
             L.qlora_status_string.argtypes = [I32]
             L.qlora_status_string.restype = ctypes.c_char_p
             L.qlora_version.argtypes = []
@@ -368,3 +391,84 @@ def qlora_linear_fwd_noalloc(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B:
                                           float(alpha), _ptr(Y), _ptr(T_save), _ptr(d_status),
                                           _stream(stream)), "qlora_linear_fwd_noalloc")
     return Y
+
+
+# ------------------------------------------------------------- LoRA dropout
+
+def qlora_workspace_bytes_dropout(M: int, N: int, K: int, r: int) -> int:
+    return int(lib().qlora_workspace_bytes_dropout(M, N, K, r))
+
+
+def qlora_lora_dropout_mask(M: int, K: int, p: float, seed: int, device="cuda", stream=None) -> torch.Tensor:
+    """The keep mask of a dropout call, uint8 [M, K] (1 = kept)."""
+    keep = torch.empty((M, K), dtype=torch.uint8, device=device)
+    _check(lib().qlora_lora_dropout_mask(M, K, float(p), int(seed), _ptr(keep), _stream(stream)),
+           "qlora_lora_dropout_mask")
+    return keep
+
+
+def qlora_linear_fwd_dropout(X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                             p: float, seed: int, Y: torch.Tensor | None = None,
+                             T_save: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                             d_status: torch.Tensor | None = None, gemm_events=None, stream=None) -> torch.Tensor:
+    """qlora_linear_fwd with LoRA dropout (rate p, mask from seed) on the adapter input."""
+    M, r = X.shape[0], A.shape[0]
+    if Y is None:
+        Y = torch.empty((M, Wq.rows), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(max(qlora_workspace_bytes_dropout(M, Wq.rows, Wq.cols, r), 16), dtype=torch.uint8,
+                                device=X.device)
+    cw = Wq.c()
+    _check(lib().qlora_linear_fwd_dropout(_ptr(X), M, ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha),
+                                          float(p), int(seed), _ptr(Y), _ptr(T_save), _ptr(workspace),
+                                          workspace.numel(), _ptr(d_status), _events(gemm_events),
+                                          _stream(stream)), "qlora_linear_fwd_dropout")
+    return Y
+
+
+def qlora_linear_bwd_dropout(dY: torch.Tensor, X: torch.Tensor, Wq: NF4Weight, A: torch.Tensor,
+                             B: torch.Tensor, alpha: float, p: float, seed: int,
+                             T_saved: torch.Tensor | None = None, dX: torch.Tensor | None = None,
+                             dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
+                             grad_dtype=torch.float32, want_dX: bool = True,
+                             workspace: torch.Tensor | None = None, d_status: torch.Tensor | None = None,
+                             gemm_events=None, stream=None):
+    """qlora_linear_bwd with the same LoRA dropout as the forward (same p and seed)."""
+    M, r = X.shape[0], A.shape[0]
+    dev = X.device
+    if want_dX and dX is None:
+        dX = torch.empty((M, Wq.cols), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((r, Wq.cols), dtype=grad_dtype, device=dev)
+    if dB is None:
+        dB = torch.empty((Wq.rows, r), dtype=grad_dtype, device=dev)
+    gdt = QLORA_F32 if dA.dtype == torch.float32 else QLORA_BF16
+    if workspace is None:
+        workspace = torch.empty(max(qlora_workspace_bytes_dropout(M, Wq.rows, Wq.cols, r), 16), dtype=torch.uint8,
+                                device=dev)
+    cw = Wq.c()
+    _check(lib().qlora_linear_bwd_dropout(_ptr(dY), _ptr(X), M, ctypes.byref(cw), _ptr(A), _ptr(B), r,
+                                          float(alpha), float(p), int(seed), _ptr(T_saved),
+                                          _ptr(dX) if want_dX else None, _ptr(dA), _ptr(dB), gdt,
+                                          _ptr(workspace), workspace.numel(), _ptr(d_status),
+                                          _events(gemm_events), _stream(stream)), "qlora_linear_bwd_dropout")
+    return dX, dA, dB
+
+
+# ------------------------------------------------------ paged optimiser state
+
+def qlora_paged_alloc(nbytes: int) -> int:
+    """Managed (pageable) device memory for optimiser state; returns the pointer."""
+    p = ctypes.c_void_p()
+    _check(lib().qlora_paged_alloc(int(nbytes), ctypes.byref(p)), "qlora_paged_alloc")
+    return int(p.value)
+
+
+def qlora_paged_free(ptr: int) -> None:
+    _check(lib().qlora_paged_free(ptr or None), "qlora_paged_free")
+
+
+def qlora_paged_prefetch(ptr: int, nbytes: int, to_device: bool = True, stream=None) -> None:
+    """Migrate [ptr, ptr + nbytes) to the current GPU, or page it out to the host."""
+    _check(lib().qlora_paged_prefetch(ptr, int(nbytes), 1 if to_device else 0, _stream(stream)),
+           "qlora_paged_prefetch")

@@ -28,8 +28,9 @@
  *   - `d_status` (nullable) is a device int the kernels OR error bits into:
  *     QLORA_DEV_NONFINITE_BIT (a non-finite weight seen by the quantiser or
  *     the merge, or a non-finite gradient seen by the Adam step) and
- *     QLORA_DEV_TIMEOUT_BIT (a pipeline wait gave up after ~2 s; the kernel
- *     then returns early and its outputs are unspecified).  The caller zeroes
+ *     QLORA_DEV_TIMEOUT_BIT (a pipeline wait gave up after ~2 s, or the
+ *     bound set by qlora_debug_set_wait_limit; the kernel then returns
+ *     early and its outputs are unspecified).  The caller zeroes
  *     it and reads it after synchronising.
  *   - Errors: a call that returns a validation error (anything but QLORA_OK
  *     and QLORA_ERR_CUDA) has enqueued nothing.  QLORA_ERR_CUDA means a
@@ -79,21 +80,31 @@ typedef struct {
  * frees them.
  *   codes       [rows, cols/2] uint8: byte j of a row holds the code of element
  *               2j in its low nibble and of element 2j+1 in its high nibble.
- *   absmax_q8   [rows*cols/64] uint8 (double_quant = 1): block b is elements
- *               64b .. 64b+63 of the row-major matrix.
- *   group_scale [ceil(rows*cols/64/256)] fp32 (double_quant = 1): group g
- *               covers blocks 256g .. 256g+255, so groups may cross rows.
+ *   absmax_q8   [rows*cols/64] uint8 (double_quant = 1 or 2): block b is
+ *               elements 64b .. 64b+63 of the row-major matrix.
+ *   group_scale [ceil(rows*cols/64/256)] fp32 (double_quant = 1 or 2): group
+ *               g covers blocks 256g .. 256g+255, so groups may cross rows.
  *   absmax_f32  [rows*cols/64] fp32 (double_quant = 0, or an optional extra
  *               output of the quantiser when non-null).
- * Block scale: double_quant ? float(absmax_q8[b]) * group_scale[b/256]
- *                           : absmax_f32[b].
+ * double_quant selects the second-level format of the block scales:
+ *   0 (QLORA_DQ_NONE): fp32 absmax per block, absmax_f32[b];
+ *   1 (QLORA_DQ_U8):   linear 8-bit, float(absmax_q8[b]) * group_scale[b/256],
+ *                      group_scale = max absmax / 255 (the learning-llms
+ *                      page's 8-bit double quantisation);
+ *   2 (QLORA_DQ_E4M3): FP8 E4M3 codes, E4M3(absmax_q8[b]) * group_scale[b/256],
+ *                      group_scale = max absmax / 448 ("QLoRA", infra.bea.ai,
+ *                      §1 subsection "Double Quantization": scales to FP8).
+ * Both 8-bit formats store 4 + 8/64 + 32/16384 = 4.127 bits per weight.
  */
+#define QLORA_DQ_NONE 0
+#define QLORA_DQ_U8 1
+#define QLORA_DQ_E4M3 2
 typedef struct {
   int64_t rows;          /* N */
   int64_t cols;          /* K, a multiple of 64 */
   int32_t blocksize;     /* must be 64 */
   int32_t group;         /* must be 256 */
-  int32_t double_quant;  /* 1: absmax_q8 + group_scale; 0: absmax_f32 */
+  int32_t double_quant;  /* QLORA_DQ_*: 1 or 2: absmax_q8 + group_scale; 0: absmax_f32 */
   int32_t reserved;      /* must be 0 */
   uint8_t* codes;
   uint8_t* absmax_q8;
@@ -125,8 +136,10 @@ void qlora_nf4_codebook(float* out16);
  * section "The mechanism": the base is quantised a single time, at load).  W: device [rows, cols], fp32 (w_dtype = QLORA_F32) or bf16.
  * Per 64-block: absmax; x = w * fp32(1/absmax); code = nearest NF4 level
  * (ties to the lower code); a block with absmax below FLT_MIN is all code 7.
- * With double_quant, per 256-block group: s = fp32(max absmax / 255),
- * q8 = min(255, rint(absmax / s)) (s = 0 and q8 = 0 when the group max is
+ * With double_quant = 1, per 256-block group: s = fp32(max absmax / 255),
+ * q8 = min(255, rint(absmax / s)); with double_quant = 2: s = fp32(max
+ * absmax / 448), q8 = the E4M3 code of fp32(absmax / s), round to nearest
+ * even, saturating at 448 (in both, s = 0 and q8 = 0 when the group max is
  * below FLT_MIN); the codes use the fp32 absmax.  out->absmax_f32 is
  * written when non-null.  A non-finite weight sets QLORA_DEV_NONFINITE_BIT;
  * the outputs are then unspecified.
@@ -193,6 +206,50 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M,
                               qlora_dtype grad_dtype, void* workspace,
                               size_t ws_bytes, int* d_status,
                               const qlora_gemm_events* events, void* stream);
+
+/*
+ * LoRA dropout ("QLoRA", infra.bea.ai, §3 "Implementation": the adapter
+ * configuration sets lora_dropout = 0.05 without defining it).  Read here as
+ * inverted dropout on the adapter's input only: the frozen path sees X,
+ * the adapter sees X * keep, kept elements scaled by 1 / (1 - p):
+ *     T  = (X * keep) A^T / (1 - p)        Y  = X W^T + s T B^T
+ *     G  = dY B                            dX = dY W^ + s ((G A) * keep) / (1 - p)
+ *     dA = s G^T (X * keep) / (1 - p)      dB = s dY^T T
+ * One mask per call from a counter-based generator, so the forward and the
+ * backward of a step regenerate the same mask from the same (p, seed):
+ * element e = m*K + k of X [M, K] is kept iff the top 32 bits of word e % 4
+ * of Philox-4x64-10 (Salmon et al., SC 2011) at counter (e / 4, 0, 0, 0),
+ * key (seed, 0), are >= ceil(p * 2^32).  0 <= p < 1 (p = 0 keeps every
+ * element: the plain layer); a p outside that range is QLORA_ERR_INVALID_ARG.
+ *
+ * qlora_workspace_bytes_dropout: workspace of the two dropout entries (the
+ * plain one plus X * keep [M, K] bf16, the frozen-path dX in fp32 [M, K] and
+ * G in fp32 [M, r]).  Host-only; 0 for an invalid shape.
+ * qlora_lora_dropout_mask: the call's keep mask into keep (device, uint8
+ * [M, K], 1 = kept, 0 = dropped), for callers and tests that need it.
+ * qlora_linear_fwd_dropout / qlora_linear_bwd_dropout: the forward and the
+ * backward above; every other argument, layout, error and determinism rule
+ * is that of qlora_linear_fwd / qlora_linear_bwd.  T_save / T_saved hold
+ * T as defined above (scaled by 1 / (1 - p)).  Under dropout the adapter
+ * term of dX cannot be folded into the fused GEMM (the mask is per element),
+ * so the GEMM writes dY W^ in fp32 and one more pass adds the masked term
+ * and rounds once to bf16.
+ */
+size_t qlora_workspace_bytes_dropout(int64_t M, int64_t N, int64_t K, int r);
+qlora_status qlora_lora_dropout_mask(int64_t M, int64_t K, double p, uint64_t seed, uint8_t* keep,
+                                     void* stream);
+qlora_status qlora_linear_fwd_dropout(const void* X, int64_t M, const qlora_nf4_weight* Wq,
+                                      const void* A, const void* B, int r, float alpha, double p,
+                                      uint64_t seed, void* Y, float* T_save, void* workspace,
+                                      size_t ws_bytes, int* d_status,
+                                      const qlora_gemm_events* events, void* stream);
+qlora_status qlora_linear_bwd_dropout(const void* dY, const void* X, int64_t M,
+                                      const qlora_nf4_weight* Wq, const void* A, const void* B,
+                                      int r, float alpha, double p, uint64_t seed,
+                                      const float* T_saved, void* dX, void* dA, void* dB,
+                                      qlora_dtype grad_dtype, void* workspace, size_t ws_bytes,
+                                      int* d_status, const qlora_gemm_events* events,
+                                      void* stream);
 
 /*
  * The same forward and backward over a dense bf16 weight W [N, K] (plain
@@ -269,6 +326,47 @@ qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16
                              int64_t step, float lr, float beta1, float beta2, float eps,
                              float weight_decay, float grad_scale, int* d_status,
                              void* stream);
+
+/*
+ * Test hooks for the bounded device waits (no counterpart on the pages).
+ * Every pipeline wait in the kernels gives up after a bound (2 s by default),
+ * sets QLORA_DEV_TIMEOUT_BIT in the call's d_status, and lets the kernel
+ * release its resources and return, so that the context stays usable.
+ *   qlora_debug_set_wait_limit: the bound in ns for the current device
+ *     (0 restores 2 s); a synchronous copy to device memory.
+ *   qlora_debug_inject_stall(on): while on, CTA 0 of every adapter-product
+ *     launch of this library (the T = X A^T, G = dY B and dA/dB products)
+ *     withholds the loads of its first pipeline stage, so that its wait
+ *     runs out; the launch then ends early with the timeout bit set and the
+ *     call's outputs unspecified.  Calls after it is switched off are
+ *     unaffected (each call clears the arrival counters it uses).
+ * Neither is for production use; both apply to kernels enqueued afterwards.
+ */
+qlora_status qlora_debug_set_wait_limit(uint64_t ns);
+qlora_status qlora_debug_inject_stall(int on);
+
+/*
+ * Paged optimiser state ("QLoRA", learning-llms page, the paragraph on paged
+ * optimizers; "QLoRA", scalata.ai, "How it works": optimiser state kept in
+ * unified memory, which the driver pages out to host RAM when a memory
+ * spike would otherwise end the run, and back in when the GPU touches it).
+ * qlora_adam_step takes any device-addressable pointers, so paged state
+ * needs no other kernel; these three calls manage it:
+ *   qlora_paged_alloc: `bytes` of CUDA managed memory into *ptr (host
+ *     pointer to the handle), preferred location the current device.  This
+ *     and qlora_paged_free are the library's only calls that allocate or
+ *     free; bytes == 0 or ptr == NULL is QLORA_ERR_INVALID_ARG.
+ *   qlora_paged_free: releases what qlora_paged_alloc returned (NULL: no-op).
+ *   qlora_paged_prefetch: enqueues on `stream` a migration of
+ *     [ptr, ptr + bytes) to the current device (to_device != 0) or to the
+ *     host (to_device == 0: paged out; the GPU's next access faults the
+ *     pages back in).  Contents are unchanged.
+ * The host may read and write the memory directly between GPU work (after
+ * synchronising), which is how a test fills and checks optimiser state.
+ */
+qlora_status qlora_paged_alloc(size_t bytes, void** ptr);
+qlora_status qlora_paged_free(void* ptr);
+qlora_status qlora_paged_prefetch(void* ptr, size_t bytes, int to_device, void* stream);
 
 /*
  * Forward without a caller workspace, for callers that cannot allocate

@@ -80,7 +80,7 @@ FAKE = 1 << 40
 
 @pytest.mark.parametrize("field,value,expect", [
     ("blocksize", 32, 2), ("group", 128, 2), ("cols", 100, 1), ("rows", 0, 1),
-    ("reserved", 1, 1), ("double_quant", 2, 1), ("codes", None, 1), ("codes", FAKE + 8, 1),
+    ("reserved", 1, 1), ("double_quant", 3, 1), ("double_quant", -1, 1), ("codes", None, 1), ("codes", FAKE + 8, 1),
 ])
 def test_quantize_rejects_bad_weight_descriptor(field, value, expect):
     w = _w(**{field: value})
@@ -135,6 +135,36 @@ def test_linear_bwd_validation():
     assert L.qlora_linear_bwd(*bad) == 6
     bad = list(args); bad[8] = FAKE + 4              # misaligned T_saved
     assert L.qlora_linear_bwd(*bad) == 1
+
+
+def test_dropout_validation():
+    # an invalid rate or a workspace sized for the plain layer is rejected
+    # before anything is enqueued (no GPU needed for these answers)
+    w = _w()
+    L = q.lib()
+    need = q.qlora_workspace_bytes_dropout(16, 256, 512, 8)
+    assert need > q.qlora_workspace_bytes(16, 256, 512, 8) + 16 * 512 * 6
+    assert q.qlora_workspace_bytes_dropout(0, 256, 512, 8) == 0
+    args = [FAKE, 16, ctypes.byref(w), FAKE, FAKE, 8, 16.0, 0.05, 7, FAKE, None, FAKE, need, None, None, None]
+    for p in (-0.01, 1.0, float("nan"), float("inf")):
+        bad = list(args); bad[7] = p
+        assert L.qlora_linear_fwd_dropout(*bad) == 1
+    bad = list(args); bad[12] = q.qlora_workspace_bytes(16, 256, 512, 8)
+    assert L.qlora_linear_fwd_dropout(*bad) == 6
+    bargs = [FAKE, FAKE, 16, ctypes.byref(w), FAKE, FAKE, 8, 16.0, 0.05, 7, None, FAKE, FAKE, FAKE, 0, FAKE,
+             need, None, None, None]
+    bad = list(bargs); bad[8] = 1.5
+    assert L.qlora_linear_bwd_dropout(*bad) == 1
+    bad = list(bargs); bad[12] = None                # dA
+    assert L.qlora_linear_bwd_dropout(*bad) == 1
+    assert L.qlora_lora_dropout_mask(16, 512, 1.0, 7, FAKE, None) == 1
+    assert L.qlora_lora_dropout_mask(16, 100, 0.1, 7, FAKE, None) == 1      # K % 64 != 0
+    assert L.qlora_lora_dropout_mask(16, 512, 0.1, 7, None, None) == 1
+
+
+def test_fp8_scale_format_sizes():
+    # E4M3 second-level scales take the same storage as the 8-bit format
+    assert q.qlora_nf4_sizes(256, 512, 2) == q.qlora_nf4_sizes(256, 512, 1)
 
 
 def test_lora_dense_validation():

@@ -40,9 +40,12 @@ def _call_noalloc(X, Wq, A, B, alpha, Y, T):
 
 @pytest.mark.parametrize("M,N,K,r", [
     (200, 264, 576, 8), (2048, 4096, 4096, 16), (96, 136, 448, 5),
-    (16, 512, 1024, 16), (1, 256, 512, 8),      # decode shapes: the weight-streaming kernel on the fixed scratch
+    (16, 512, 1024, 16), (1, 8192, 512, 8),     # decode shapes: the weight-streaming kernel on the fixed scratch
 ])
 def test_noalloc_forward_matches_workspace_forward_twice(M, N, K, r):
+    # (every case has >= 8192 outputs: the bf16 rounding of Y alone gives a
+    # relative error near 1.7e-3 on average, and on a few hundred outputs it
+    # can exceed the 2e-3 bar by chance)
     # The entry point runs the same kernels with the same plans as the
     # workspace forward, only on other scratch memory, so Y and T must be
     # bit-identical to it; both are also held to the oracle's tolerance.
