@@ -249,7 +249,9 @@ class Layer:
         q, alpha = self.q, self.wl.alpha
         comp = torch.cuda.current_stream()
         ev[0].record(comp)
-        s_h2d.wait_event(ev[0])
+        fork = torch.cuda.Event()      # an ordinary event for the fork: the timing one may be a graph node
+        fork.record(comp)
+        s_h2d.wait_event(fork)
         ready_x, ready_dy = {}, {}
         with torch.cuda.stream(s_h2d):
             for p in self.proj:
@@ -299,6 +301,16 @@ class Layer:
         f = [2 * self.M * p["N"] * p["K"] + 2 * self.M * r * p["N"] for p in self.proj]
         b = [2 * self.M * p["N"] * p["K"] + 2 * self.M * r * p["K"] for p in reversed(self.proj)]
         return f + b
+
+
+def capture_graph(fn):
+    """One CUDA graph of everything fn enqueues (the library's calls validate
+    on the host and only enqueue, so they can be captured).  Events fn records
+    must already exist (record them once outside the capture)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
 
 
 def flush_l2(buf):
@@ -369,6 +381,18 @@ def run_ours(args):
                 for _ in range(2 * nproj)] for _ in range(args.steps)]
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
+    graphs = None
+    if not args.no_graph:
+        # one graph per timed step (each with its own GEMM timing events):
+        # a replay launches the step's 35 kernels and memsets without the
+        # host's per-launch gaps between them
+        for evs in gemm_ev:
+            for a, b in evs:
+                a.record(); b.record()
+        torch.cuda.synchronize()
+        graphs = [capture_graph(lambda i=i: layer.step(gemm_events=list(gemm_ev[i]))) for i in range(args.steps)]
+        graphs[0].replay()
+        torch.cuda.synchronize()
     clocks = ClockSampler(local, args.clock_log)
     clocks.start()
     time.sleep(0.3)
@@ -377,7 +401,10 @@ def run_ours(args):
     for i in range(args.steps):
         flush_l2(l2buf)
         step_ev[i][0].record()
-        layer.step(gemm_events=list(gemm_ev[i]))
+        if graphs is not None:
+            graphs[i].replay()
+        else:
+            layer.step(gemm_events=list(gemm_ev[i]))
         allreduce_grads()
         step_ev[i][1].record()
     torch.cuda.synchronize()
@@ -408,14 +435,29 @@ def run_ours(args):
         hostdB = [torch.empty_like(p["dB"], device="cpu").pin_memory() for p in layer.proj]
         h2d = sum(t.numel() * t.element_size() for t in list(hostX.values()) + hostdY)
         d2h = sum(t.numel() * t.element_size() for t in hostdA + hostdB)
-        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        # external: recorded as event nodes when captured into a graph
+        e_ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
                 for _ in range(args.steps)]
         s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        egraphs = None
+        if not args.no_graph and world == 1:
+            # the whole end-to-end step -- copies in, kernels, copies out --
+            # as one graph per timed step (NCCL stays outside graphs)
+            for a, b in e_ev:
+                a.record(); b.record()
+            torch.cuda.synchronize()
+            egraphs = [capture_graph(lambda i=i: layer.step_e2e(hostX, hostdY, hostdA, hostdB, s_h2d, s_d2h,
+                                                                e_ev[i]))
+                       for i in range(args.steps)]
         barrier()
         torch.cuda.synchronize()
         for i in range(args.steps):
             flush_l2(l2buf)
-            layer.step_e2e(hostX, hostdY, hostdA, hostdB, s_h2d, s_d2h, e_ev[i], allreduce_grads if world > 1 else None)
+            if egraphs is not None:
+                egraphs[i].replay()
+            else:
+                layer.step_e2e(hostX, hostdY, hostdA, hostdB, s_h2d, s_d2h, e_ev[i],
+                               allreduce_grads if world > 1 else None)
         torch.cuda.synchronize()
         barrier()
         e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), world, dev)
@@ -452,6 +494,8 @@ def run_ours(args):
                    "inputs": "q/k/v read one X, gate/up another (as in the decoder layer)",
                    "weights": "NF4 double-quant, block 64, group 256",
                    "flops_per_step": step_flops(), "l2": "flushed between timed steps",
+                   "launch": "each timed step replays a CUDA graph of its library calls" if graphs is not None
+                             else "library calls launched one by one",
                    "parallelism": f"dp{world}"},
         "roofline": {"bound": "tensor", "kernel": "k_gemm_nf4_pair (fused NF4 dequant + 2-SM tcgen05 GEMM)",
                      "achieved": round(g_achieved, 2), "peak": round(peak_burst, 1), "unit": "TFLOP/s",
@@ -1056,6 +1100,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps call by call instead of replaying a CUDA graph per step")
     ap.add_argument("--no-cpu-legs", action="store_true",
                     help="time only the oracle's layer-step sample, not its codec / decode / quantise legs")
     ap.add_argument("--clock-log", default=None,

@@ -112,6 +112,16 @@ int sm_count() {
   return v;
 }
 
+// Record a caller's timing event on the stream.  Under stream capture the
+// record becomes an event node of the graph (an ordinary cudaEventRecord
+// would only add an ordering dependency), so that every replay records it.
+cudaError_t record_event(cudaEvent_t e, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    return cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+  return cudaEventRecord(e, st);
+}
+
 qlora_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
@@ -391,7 +401,7 @@ qlora_status launch_gemm(int mode, const CUtensorMap& tact, const CUtensorMap& t
                          const CUtensorMap& tlb, const GemmArgs& a, const qlora_gemm_events* ev,
                          cudaStream_t st) {
   dim3 grid(static_cast<unsigned>(cdiv(a.out_cols, kGemmBN)), static_cast<unsigned>(cdiv(a.M, kGemmBM)));
-  if (ev && ev->gemm_start && cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_start), st) != cudaSuccess)
+  if (ev && ev->gemm_start && record_event(static_cast<cudaEvent_t>(ev->gemm_start), st) != cudaSuccess)
     return QLORA_ERR_CUDA;
   if (mode == kModeFwd)
     k_gemm_nf4<kModeFwd><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tact, tcodes, tla, tlb, a);
@@ -399,7 +409,7 @@ qlora_status launch_gemm(int mode, const CUtensorMap& tact, const CUtensorMap& t
     k_gemm_nf4<kModeDx><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tact, tcodes, tla, tlb, a);
   qlora_status rc = check_launch();
   if (rc == QLORA_OK && ev && ev->gemm_end &&
-      cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_end), st) != cudaSuccess)
+      record_event(static_cast<cudaEvent_t>(ev->gemm_end), st) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return rc;
 }
@@ -459,7 +469,7 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   a.status = status;
   if (!pair) return launch_gemm(mode, tact, tcodes, tla, tlb, a, ev, cs);
 
-  if (ev && ev->gemm_start && cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_start), cs) != cudaSuccess)
+  if (ev && ev->gemm_start && record_event(static_cast<cudaEvent_t>(ev->gemm_start), cs) != cudaSuccess)
     return QLORA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * cdiv(a.out_cols, 256)), static_cast<unsigned>(cdiv(d.M, 256)));
@@ -484,7 +494,7 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
     cudaGetLastError();
     return QLORA_ERR_CUDA;
   }
-  if (ev && ev->gemm_end && cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_end), cs) != cudaSuccess)
+  if (ev && ev->gemm_end && record_event(static_cast<cudaEvent_t>(ev->gemm_end), cs) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return QLORA_OK;
 }
@@ -525,7 +535,7 @@ qlora_status run_gemv(const void* X, const void* A, const qlora_nf4_weight* Wq, 
   a.units = units;
   a.status = status;
   if (cudaMemsetAsync(a.cnt, 0, static_cast<size_t>(tiles + 2) * 4, cs) != cudaSuccess) return QLORA_ERR_CUDA;
-  if (ev && ev->gemm_start && cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_start), cs) != cudaSuccess)
+  if (ev && ev->gemm_start && record_event(static_cast<cudaEvent_t>(ev->gemm_start), cs) != cudaSuccess)
     return QLORA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -540,7 +550,7 @@ qlora_status run_gemv(const void* X, const void* A, const qlora_nf4_weight* Wq, 
   if (cudaLaunchKernelEx(&cfg, k_gemv_nf4, tx, tc, a) != cudaSuccess) return QLORA_ERR_CUDA;
   qlora_status rc = check_launch();
   if (rc == QLORA_OK && ev && ev->gemm_end &&
-      cudaEventRecord(static_cast<cudaEvent_t>(ev->gemm_end), cs) != cudaSuccess)
+      record_event(static_cast<cudaEvent_t>(ev->gemm_end), cs) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return rc;
 }

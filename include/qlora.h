@@ -68,7 +68,8 @@ typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
  * (cudaEvent_t passed as void*) that the call records on `stream` right
  * before and right after its fused NF4 GEMM launch, so that a caller can
  * time that kernel alone.  The struct and either member may be NULL; the
- * events are owned by the caller.
+ * events are owned by the caller.  Under stream capture the records become
+ * event nodes of the graph, so every replay records them.
  */
 typedef struct {
   void* gemm_start;
