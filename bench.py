@@ -164,6 +164,12 @@ def max_over_ranks(x, world, device):
 X_SOURCE = {"q": "q", "k": "q", "v": "q", "o": "o", "gate": "gate", "up": "gate", "down": "down"}
 
 
+# Projections of a decoder layer that do not depend on one another: q, k and
+# v read the same input, and so do gate and up.  o needs attention's output
+# and down the gated MLP product, so each of those runs alone.
+CONCURRENT_GROUPS = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))
+
+
 class Layer:
     """Seven NF4 projections of one layer, resident on the device (q/k/v and
     gate/up share their input tensor, as in the model)."""
@@ -199,6 +205,11 @@ class Layer:
             self.proj.append(p)
         ws = max(q.qlora_workspace_bytes(M, p["N"], p["K"], wl.r) for p in self.proj)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        # a workspace per projection, for projections that run concurrently
+        self.wss = [torch.empty(q.qlora_workspace_bytes(M, p["N"], p["K"], wl.r), dtype=torch.uint8, device=device)
+                    for p in self.proj]
+        self.groups = [[index[n] for n in g] for g in CONCURRENT_GROUPS if all(n in index for n in g)]
+        self.side = [torch.cuda.Stream(device=device) for _ in range(max(len(g) for g in self.groups))]
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def quantize_all(self, events=None):
@@ -213,6 +224,48 @@ class Layer:
     def drop_source_weights(self):
         for p in self.proj:
             p.pop("W_tmp", None)
+
+    def _fwd(self, i, ev, ws):
+        p = self.proj[i]
+        self.q.qlora_linear_fwd(p["X"], p["Wq"], p["A"], p["B"], self.wl.alpha, Y=p["Y"], T_save=p["T"],
+                                workspace=ws, d_status=self.status, gemm_events=ev)
+
+    def _bwd(self, i, ev, ws):
+        p = self.proj[i]
+        self.q.qlora_linear_bwd(p["dY"], p["X"], p["Wq"], p["A"], p["B"], self.wl.alpha, T_saved=p["T"],
+                                dX=p["dX"], dA=p["dA"], dB=p["dB"], workspace=ws, d_status=self.status,
+                                gemm_events=ev)
+
+    def _group(self, idx, fn, evs):
+        """Run fn(i, ev, ws) for the projections idx: alone on the current
+        stream, or each on a side stream forked from and joined back into it."""
+        main = torch.cuda.current_stream()
+        if len(idx) == 1:
+            fn(idx[0], evs.get(idx[0]), self.wss[idx[0]])
+            return
+        fork = torch.cuda.Event()
+        fork.record(main)
+        joins = []
+        for s, i in zip(self.side, idx):
+            s.wait_event(fork)
+            with torch.cuda.stream(s):
+                fn(i, evs.get(i), self.wss[i])
+                e = torch.cuda.Event()
+                e.record(s)
+            joins.append(e)
+        for e in joins:
+            main.wait_event(e)
+
+    def step_concurrent(self, gemm_events=None):
+        """The step with independent projections overlapped (CONCURRENT_GROUPS):
+        forward group by group, then backward in reverse group order."""
+        n = len(self.proj)
+        fev = {i: gemm_events[i] for i in range(n)} if gemm_events else {}
+        bev = {i: gemm_events[n + (n - 1 - i)] for i in range(n)} if gemm_events else {}
+        for g in self.groups:
+            self._group(g, self._fwd, fev)
+        for g in reversed(self.groups):
+            self._group(list(reversed(g)), self._bwd, bev)
 
     def step(self, gemm_events=None):
         """Forward of all 7 projections, then backward in reverse order."""
@@ -390,7 +443,8 @@ def run_ours(args):
             for a, b in evs:
                 a.record(); b.record()
         torch.cuda.synchronize()
-        graphs = [capture_graph(lambda i=i: layer.step(gemm_events=list(gemm_ev[i]))) for i in range(args.steps)]
+        stepfn = layer.step_concurrent if args.concurrent else layer.step
+        graphs = [capture_graph(lambda i=i: stepfn(gemm_events=list(gemm_ev[i]))) for i in range(args.steps)]
         graphs[0].replay()
         torch.cuda.synchronize()
     clocks = ClockSampler(local, args.clock_log)
@@ -1100,6 +1154,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--concurrent", action="store_true",
+                    help="overlap independent projections (q/k/v, gate/up) on side streams inside the step graph")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps call by call instead of replaying a CUDA graph per step")
     ap.add_argument("--no-cpu-legs", action="store_true",

@@ -107,6 +107,36 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is incomplete is
+// suspended (issuing nothing) for up to `ns` or until the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait built on the hinted try_wait (for a thread whose polling
+// would take issue slots from busy warps on its scheduler).
+__device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               int* status, uint32_t ns) {
+  if (mbar_try_wait_hint(bar, parity, ns)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait_hint(bar, parity, ns)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > qlora_wait_limit()) {
+      *abort_flag = 1;
+      if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Bounded wait for a role that is not on the critical path and may wait a
 // long time (a producer ahead of its consumers, an epilogue waiting for a
 // whole tile): it sleeps `ns` between polls instead of spinning, so that it
