@@ -48,7 +48,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one fused-GEMM launch (gate forward) from the ncu capture
 # summarised in profiles/k_gemm_nf4_pair_fwd_gate_m2048.md; None once the
 # kernel changes and until it is captured again.
-GEMM_TRAFFIC_BYTES = 48.26e6
+GEMM_TRAFFIC_BYTES = 48.94e6
 
 
 def step_flops(wl=WL, M=None) -> float:
@@ -434,18 +434,23 @@ def run_ours(args):
                 for _ in range(2 * nproj)] for _ in range(args.steps)]
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
-    graphs = None
+    graphs = seq_graphs = None
+    concurrent = not args.sequential and not args.no_graph
     if not args.no_graph:
-        # one graph per timed step (each with its own GEMM timing events):
-        # a replay launches the step's 35 kernels and memsets without the
-        # host's per-launch gaps between them
+        # one graph per timed step: a replay launches the step's 35 kernels
+        # and memsets without the host's per-launch gaps between them.  The
+        # headline step overlaps the layer's independent projections
+        # (q/k/v, gate/up); the roofline pass replays the same calls in
+        # sequence, each graph with its own GEMM timing events, so that each
+        # fused-GEMM launch is timed alone
         for evs in gemm_ev:
             for a, b in evs:
                 a.record(); b.record()
         torch.cuda.synchronize()
-        stepfn = layer.step_concurrent if args.concurrent else layer.step
-        graphs = [capture_graph(lambda i=i: stepfn(gemm_events=list(gemm_ev[i]))) for i in range(args.steps)]
+        seq_graphs = [capture_graph(lambda i=i: layer.step(gemm_events=list(gemm_ev[i]))) for i in range(args.steps)]
+        graphs = ([capture_graph(layer.step_concurrent) for _ in range(args.steps)] if concurrent else seq_graphs)
         graphs[0].replay()
+        seq_graphs[0].replay()
         torch.cuda.synchronize()
     clocks = ClockSampler(local, args.clock_log)
     clocks.start()
@@ -463,8 +468,20 @@ def run_ours(args):
         step_ev[i][1].record()
     torch.cuda.synchronize()
     barrier()
-    clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    seq_ms = step_ms
+    if concurrent:
+        # roofline pass: the same steps in sequence (L2 flushed likewise)
+        seq_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush_l2(l2buf)
+            seq_ev[i][0].record()
+            seq_graphs[i].replay()
+            seq_ev[i][1].record()
+        torch.cuda.synchronize()
+        seq_ms = [a.elapsed_time(b) for a, b in seq_ev]
+    clk = clocks.stop()
     gemm_ms = [[a.elapsed_time(b) for a, b in evs] for evs in gemm_ev]
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     assert layer.status.item() == 0, f"device status {layer.status.item()}"
@@ -478,7 +495,7 @@ def run_ours(args):
     g_achieved = sum(gflops) * args.steps / g_time / 1e12
     peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     peak_burst = float(peaks.get("bf16_tflops"))
-    gemm_share = g_time * 1e3 / sum(step_ms)
+    gemm_share = g_time * 1e3 / sum(seq_ms)
 
     # ---- end to end through host buffers (pinned), copies inside the timed region
     e2e = None
@@ -548,8 +565,11 @@ def run_ours(args):
                    "inputs": "q/k/v read one X, gate/up another (as in the decoder layer)",
                    "weights": "NF4 double-quant, block 64, group 256",
                    "flops_per_step": step_flops(), "l2": "flushed between timed steps",
-                   "launch": "each timed step replays a CUDA graph of its library calls" if graphs is not None
-                             else "library calls launched one by one",
+                   "launch": ("each timed step replays a CUDA graph of its library calls; independent "
+                              "projections (q/k/v, then gate/up; their backward likewise) overlap on side "
+                              "streams, o and down run alone" if concurrent else
+                              "each timed step replays a CUDA graph of its library calls, in sequence")
+                             if graphs is not None else "library calls launched one by one",
                    "parallelism": f"dp{world}"},
         "roofline": {"bound": "tensor", "kernel": "k_gemm_nf4_pair (fused NF4 dequant + 2-SM tcgen05 GEMM)",
                      "achieved": round(g_achieved, 2), "peak": round(peak_burst, 1), "unit": "TFLOP/s",
@@ -560,6 +580,9 @@ def run_ours(args):
                      "frac_of_sustained_peak": round(g_achieved / peak_sus, 4),
                      "launches": g_launches, "avg_launch_us": round(g_time / g_launches * 1e6, 2),
                      "share_of_step": round(gemm_share, 4),
+                     "timed_on": ("a sequential replay of the same step graphs right after the timed steps "
+                                  f"({round(sum(seq_ms) / len(seq_ms), 4)} ms per step), each launch alone"
+                                  if concurrent else "the timed steps"),
                      # DRAM bytes (read + write) of one launch, from the ncu capture in
                      # profiles/k_gemm_nf4_pair_fwd_gate_m2048.md (gate forward,
                      # 2048 x 11008 x 4096); its algorithmic bytes are 85.1 MB, most of
@@ -633,36 +656,74 @@ def _layer_tensors(wl, L, M, dev, x_shared=True):
     return out
 
 
-def _model_step(q, wl, nf4, acts, bufs, ws, status, layers):
-    """Forward through every projection of `layers`, then backward in reverse."""
+def run_concurrent(idx, fn, side):
+    """fn(i) for the projections idx: alone on the current stream, or each on a
+    side stream forked from and joined back into it."""
+    main = torch.cuda.current_stream()
+    if len(idx) == 1:
+        fn(idx[0])
+        return
+    fork = torch.cuda.Event()
+    fork.record(main)
+    joins = []
+    for st, i in zip(side, idx):
+        st.wait_event(fork)
+        with torch.cuda.stream(st):
+            fn(i)
+            e = torch.cuda.Event()
+            e.record(st)
+        joins.append(e)
+    for e in joins:
+        main.wait_event(e)
+
+
+def _model_step(q, wl, nf4, acts, bufs, wss, status, layers, side):
+    """Forward through every projection of `layers`, then backward in reverse;
+    within a layer the independent projections (CONCURRENT_GROUPS) overlap."""
+    index = {n: i for i, (n, _, _) in enumerate(wl.shapes)}
+    groups = [[index[n] for n in g] for g in CONCURRENT_GROUPS if all(n in index for n in g)]
+
+    def fwd(L, i):
+        a = acts[L][i]
+        q.qlora_linear_fwd(a["X"], nf4[L][i], a["A"], a["B"], wl.alpha, Y=bufs[i]["Y"], T_save=a["T"],
+                           workspace=wss[i], d_status=status)
+
+    def bwd(L, i):
+        a = acts[L][i]
+        q.qlora_linear_bwd(a["dY"], a["X"], nf4[L][i], a["A"], a["B"], wl.alpha, T_saved=a["T"],
+                           dX=bufs[i]["dX"], dA=a["dA"], dB=a["dB"], workspace=wss[i], d_status=status)
+
     for L in layers:
-        for i in range(len(wl.shapes)):
-            a = acts[L][i]
-            q.qlora_linear_fwd(a["X"], nf4[L][i], a["A"], a["B"], wl.alpha, Y=bufs[i]["Y"], T_save=a["T"],
-                               workspace=ws, d_status=status)
+        for g in groups:
+            run_concurrent(g, lambda i: fwd(L, i), side)
     for L in reversed(layers):
-        for i in reversed(range(len(wl.shapes))):
-            a = acts[L][i]
-            q.qlora_linear_bwd(a["dY"], a["X"], nf4[L][i], a["A"], a["B"], wl.alpha, T_saved=a["T"],
-                               dX=bufs[i]["dX"], dA=a["dA"], dB=a["dB"], workspace=ws, d_status=status)
+        for g in reversed(groups):
+            run_concurrent(list(reversed(g)), lambda i: bwd(L, i), side)
 
 
 def _time_model_step(q, wl, nf4, acts, M, dev, layers, steps, warmup):
+    """The whole-model step captured once as a CUDA graph and replayed."""
     bufs = [dict(Y=torch.empty((M, N), dtype=torch.bfloat16, device=dev),
                  dX=torch.empty((M, K), dtype=torch.bfloat16, device=dev)) for (_, N, K) in wl.shapes]
-    ws = torch.empty(max(q.qlora_workspace_bytes(M, N, K, wl.r) for (_, N, K) in wl.shapes),
-                     dtype=torch.uint8, device=dev)
+    wss = [torch.empty(q.qlora_workspace_bytes(M, N, K, wl.r), dtype=torch.uint8, device=dev)
+           for (_, N, K) in wl.shapes]
+    side = [torch.cuda.Stream(device=dev) for _ in range(max(len(g) for g in CONCURRENT_GROUPS))]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    for _ in range(warmup):
-        _model_step(q, wl, nf4, acts, bufs, ws, status, layers)
+    run = lambda: _model_step(q, wl, nf4, acts, bufs, wss, status, layers, side)
+    run()                                  # eager once (first-use costs), then capture
     torch.cuda.synchronize()
-    ms = time_events(lambda: _model_step(q, wl, nf4, acts, bufs, ws, status, layers), steps)
+    g = capture_graph(run)
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    ms = time_events(g.replay, steps)
     torch.cuda.synchronize()
     assert int(status.item()) == 0, "device status set during a config workload"
     t = statistics.median(ms)
     flops = len(layers) * step_flops(wl, M)
     return {"value": round(flops / (t * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(t, 3),
-            "tokens": M, "layers": len(layers), "flops_per_step": flops, "steps": steps, "warmup": warmup}
+            "tokens": M, "layers": len(layers), "flops_per_step": flops, "steps": steps, "warmup": warmup,
+            "launch": "one CUDA graph per step; q/k/v and gate/up overlap within each layer"}
 
 
 def config_workloads(q, dev, hbm):
@@ -1154,8 +1215,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--concurrent", action="store_true",
-                    help="overlap independent projections (q/k/v, gate/up) on side streams inside the step graph")
+    ap.add_argument("--sequential", action="store_true",
+                    help="run the step's projections one after another (default: q/k/v and gate/up overlap)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps call by call instead of replaying a CUDA graph per step")
     ap.add_argument("--no-cpu-legs", action="store_true",
