@@ -59,6 +59,12 @@ def _check(n, seed, grad_dtype=torch.float32, t=4, lr=1e-3, betas=(0.9, 0.999), 
     assert np.all(np.abs(gv - ov) <= 1e-6 * np.abs(ov) + 1e-37), "v"
     assert np.all(np.abs(gt - ot) <= 1e-6 * np.abs(theta.double().numpy()) + 1e-5 * lr), "master"
     assert torch.equal(param.cpu(), dm.cpu().to(torch.bfloat16)), "bf16 copy is not RNE of the master"
+    # and against the oracle's own master: the bf16 copy is within one bf16
+    # step of it (the two masters differ by fp32 rounding, which may flip the
+    # rounding of a value next to a bf16 midpoint, never by more)
+    pb = param.cpu().double().numpy()
+    ulp = np.abs(ot) * 2.0 ** -7 + 1e-37
+    assert np.all(np.abs(pb - ot) <= ulp), "bf16 copy vs the oracle's master"
     return dm, dmm, dv, param
 
 
