@@ -12,41 +12,71 @@ namespace qlora {
 
 constexpr int kQuantThreads = 256;  // one CTA per 256-block group
 
-// The 8 weights a thread holds per block, kept as loaded (a bf16 uint4
-// is 4 registers instead of 8 floats) and widened only when encoded.
-template <typename T> struct Raw8;
-template <> struct Raw8<__nv_bfloat16> { uint4 u; };
-template <> struct Raw8<float> { float4 a, b; };
-__device__ __forceinline__ Raw8<__nv_bfloat16> load_raw8(const __nv_bfloat16* p) {
-  return {__ldg(reinterpret_cast<const uint4*>(p))};
+// The 16 weights a thread holds per block, kept as loaded (bf16: two uint4,
+// 8 registers instead of 16 floats) and widened only when encoded.
+template <typename T> struct Raw16;
+template <> struct Raw16<__nv_bfloat16> { uint4 a, b; };
+template <> struct Raw16<float> { float4 a, b, c, d; };
+__device__ __forceinline__ Raw16<__nv_bfloat16> load_raw16(const __nv_bfloat16* p) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  return {__ldg(q), __ldg(q + 1)};
 }
-__device__ __forceinline__ Raw8<float> load_raw8(const float* p) {
-  return {__ldg(reinterpret_cast<const float4*>(p)), __ldg(reinterpret_cast<const float4*>(p) + 1)};
+__device__ __forceinline__ Raw16<float> load_raw16(const float* p) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+  return {__ldg(q), __ldg(q + 1), __ldg(q + 2), __ldg(q + 3)};
 }
-__device__ __forceinline__ void widen8(const Raw8<__nv_bfloat16>& r, float (&v)[8]) {
-  const uint32_t w[4] = {r.u.x, r.u.y, r.u.z, r.u.w};
+__device__ __forceinline__ void widen16(const Raw16<__nv_bfloat16>& r, float (&v)[16]) {
+  const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 8; ++i) {
     v[2 * i] = __uint_as_float(w[i] << 16);
     v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
 }
-__device__ __forceinline__ void widen8(const Raw8<float>& r, float (&v)[8]) {
-  v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
-  v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
+__device__ __forceinline__ void widen16(const Raw16<float>& r, float (&v)[16]) {
+  const float4 q[4] = {r.a, r.b, r.c, r.d};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[4 * i] = q[i].x; v[4 * i + 1] = q[i].y; v[4 * i + 2] = q[i].z; v[4 * i + 3] = q[i].w;
+  }
+}
+// The largest |weight| of the 16 as a binary32 bit pattern.  Integer order
+// of sign-cleared patterns is magnitude order, with inf and NaN patterns
+// above every finite value; bf16 pairs are compared two at a time as
+// 16-bit lanes, then widened.
+__device__ __forceinline__ uint32_t mag_bits16(const Raw16<__nv_bfloat16>& r) {
+  const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+  return max(m & 0xFFFFu, m >> 16) << 16;
+}
+__device__ __forceinline__ uint32_t mag_bits16(const Raw16<float>& r) {
+  const float4 q[4] = {r.a, r.b, r.c, r.d};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = max(m, __float_as_uint(q[i].x) & 0x7FFFFFFFu);
+    m = max(m, __float_as_uint(q[i].y) & 0x7FFFFFFFu);
+    m = max(m, __float_as_uint(q[i].z) & 0x7FFFFFFFu);
+    m = max(m, __float_as_uint(q[i].w) & 0x7FFFFFFFu);
+  }
+  return m;
 }
 
 // Nearest NF4 level of a normalised weight: code = #{i : x > t_i}, from the
-// cell table (nf4_constants.cuh): cell = rint(32 x + 32.5), found with one
-// fused multiply-add and the 1.5 * 2^23 rounding trick (the sum's low
-// mantissa bits are the integer), then one compare against the cell's
-// threshold.  The index is clamped to the table (a NaN x, from a block with
-// an infinite absmax, reads the last cell; such blocks are flagged).
-__device__ __forceinline__ uint32_t nf4_encode(float x, const uint2* s_cell) {
-  const float y = __fadd_rn(__fmaf_rn(x, 32.0f, 32.5f), 12582912.0f);
-  const uint32_t idx = min(static_cast<uint32_t>(__float_as_int(y)) - 0x4B400000u, 65u);
-  const uint2 e = s_cell[idx];
-  return e.y + ((x > __uint_as_float(e.x)) ? 1u : 0u);
+// cell table (nf4_constants.cuh): cell = rint(16 x + 16), found with one
+// fused multiply-add whose addend 1.5 * 2^23 + 16 leaves the rounded sum's
+// low mantissa bits equal to the integer, then one compare against the
+// cell's threshold.  Both table reads are 4-byte loads from the same
+// address register.  The index is clamped to the table (a NaN x, from a
+// block with an infinite absmax, reads the last cell; such blocks are
+// flagged).
+__device__ __forceinline__ uint32_t nf4_encode(float x, const NF4CellTable* s_cell) {
+  const float y = __fmaf_rn(x, 16.0f, 12582928.0f);
+  const uint32_t idx = min(static_cast<uint32_t>(__float_as_int(y)) - 0x4B400000u, static_cast<uint32_t>(kNF4Cells - 1));
+  const float thr = s_cell->thr[idx];
+  return s_cell->base[idx] + ((x > thr) ? 1u : 0u);
 }
 
 // E4M3 code of a non-negative float: round to nearest even, values above
@@ -58,68 +88,65 @@ __device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
   return static_cast<uint32_t>(r) & 0xFFu;
 }
 
-// K1.  Grid: one CTA per group of 256 blocks (16384 weights).  Eight threads
-// share a 64-weight block (8 weights each, one 16-byte load of bf16), so a
-// warp reads 4 whole blocks = 512 contiguous bytes and writes 128 contiguous
-// bytes of codes.  The block absmax is a warp-shuffle max over the 8 lanes.
-// All 8 of a thread's loads are issued before any is used and are kept as
-// loaded (32 registers for bf16), which leaves room for 5 CTAs per SM: with
-// 8 x 16 B in flight per thread that is 160 KB per SM (HBM needs tens of KB
-// per SM in flight).  The encoding is ~11 instructions per weight.
+// K1.  Grid: one CTA per group of 256 blocks (16384 weights).  Four threads
+// share a 64-weight block (16 weights each, two 16-byte loads of bf16), so a
+// warp reads 8 whole blocks = 1 KB contiguous and writes 256 contiguous
+// bytes of codes.  The block absmax is a shuffle max over the 4 lanes; the
+// per-block work (shuffles, reciprocal, checks, stores) is spread over 16
+// weights per thread.  All 4 of a thread's block loads are issued before
+// any is used and are kept as loaded (32 registers for bf16); 4 CTAs per SM
+// keep 128 B per thread, 128 KB per SM, in flight.
+// The encoding is ~10 instructions per weight.
 template <typename T>
-__global__ void __launch_bounds__(kQuantThreads, sizeof(T) == 2 ? 5 : 3)
+__global__ void __launch_bounds__(kQuantThreads, sizeof(T) == 2 ? 4 : 3)
     k_quantize_nf4(const T* __restrict__ w, int64_t nblocks, int dq, uint8_t* __restrict__ codes,
                    uint8_t* __restrict__ q8, float* __restrict__ s2,
                    float* __restrict__ absmax_out, int* status) {
-  __shared__ uint2 s_cell[66];
+  __shared__ NF4CellTable s_cell;
   __shared__ float s_absmax[256];
   __shared__ float s_wmax[kQuantThreads / 32];
   const int tid = threadIdx.x;
-  if (tid < 66) s_cell[tid] = make_uint2(__float_as_uint(c_nf4_cells.c[tid].thr), c_nf4_cells.c[tid].base);
+  if (tid < kNF4Cells) {
+    s_cell.thr[tid] = c_nf4_cells.thr[tid];
+    s_cell.base[tid] = c_nf4_cells.base[tid];
+  }
 
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * 256;
   const int nb = static_cast<int>((nblocks - b0) < 256 ? (nblocks - b0) : 256);
-  const int sub = tid & 7;
+  const int sub = tid & 3;   // weights 16 sub .. 16 sub + 15 of the block
   bool nonfinite = false;
 
-  Raw8<T> raw[8];
+  Raw16<T> raw[4];
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int lb = it * 32 + (tid >> 3);
-    if (lb < nb) raw[it] = load_raw8(w + (b0 + lb) * 64 + sub * 8);
+  for (int it = 0; it < 4; ++it) {
+    const int lb = it * 64 + (tid >> 2);
+    if (lb < nb) raw[it] = load_raw16(w + (b0 + lb) * 64 + sub * 16);
   }
   __syncthreads();   // the cell table is in shared memory
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int lb = it * 32 + (tid >> 3);
+  for (int it = 0; it < 4; ++it) {
+    const int lb = it * 64 + (tid >> 2);
     const bool valid = lb < nb;
-    const int64_t b = b0 + lb;
-    float v[8];
-    widen8(raw[it], v);
-    uint32_t mbits = 0;
-    if (valid) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mbits = max(mbits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
-    }
-    // max over the 8 lanes of the block (integer order = magnitude order,
-    // with inf/NaN patterns above every finite value)
+    uint32_t mbits = valid ? mag_bits16(raw[it]) : 0u;
     mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, 1));
     mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, 2));
-    mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, 4));
     if (!valid) continue;
     if (mbits >= 0x7F800000u) nonfinite = true;
     const float absmax = __uint_as_float(mbits);
-    uint32_t word;
+    uint2 word;
     if (!(absmax >= FLT_MIN)) {
-      word = 0x77777777u;  // zero (or subnormal) block: every weight is code 7
+      word = make_uint2(0x77777777u, 0x77777777u);  // zero (or subnormal) block: every weight is code 7
     } else {
       const float inv = __frcp_rn(absmax);
-      word = 0;
+      float v[16];
+      widen16(raw[it], v);
+      uint32_t h[2] = {0, 0};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) word |= nf4_encode(__fmul_rn(v[i], inv), s_cell) << (4 * i);
+      for (int i = 0; i < 16; ++i) h[i >> 3] |= nf4_encode(__fmul_rn(v[i], inv), &s_cell) << (4 * (i & 7));
+      word = make_uint2(h[0], h[1]);
     }
-    reinterpret_cast<uint32_t*>(codes)[b * 8 + sub] = word;
+    reinterpret_cast<uint2*>(codes)[(b0 + lb) * 4 + sub] = word;
     if (sub == 0) s_absmax[lb] = absmax;
   }
   if (nonfinite && status) atomicOr(status, QLORA_DEV_NONFINITE);

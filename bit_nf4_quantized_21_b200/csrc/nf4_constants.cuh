@@ -57,51 +57,54 @@ __constant__ float c_nf4_level[16] = {QLORA_NF4_LEVELS};
 __constant__ float c_nf4_threshold[15] = {QLORA_NF4_THRESHOLDS};
 
 // The encoder's cell table.  x in [-1, 1] (|x| may exceed 1 by a rounding)
-// is cut into 66 cells of width 1/32: cell i holds x in
-// [(i - 33)/32, (i - 32)/32), i = rint(32 x + 32.5).  Each cell holds at
-// most one threshold (the thresholds are >= 0.08 apart), so
+// is cut into 33 cells of width 1/16 centred on the multiples of 1/16:
+// cell i = rint(16 x + 16) holds x in [(2i - 33)/32, (2i - 31)/32].  Each
+// cell holds at most one threshold (consecutive thresholds are >= 0.08
+// apart), so
 //   #{j : x > t_j} = base_i + (x > thr_i)
-// with base_i = #{j : t_j < (i - 33)/32} and thr_i the cell's threshold
+// with base_i = #{j : t_j < (2i - 33)/32} and thr_i the cell's threshold
 // (2.0, above every x, when it has none).  Every threshold lies >= 1.6e-3
-// from a cell edge, far more than the ~1.2e-7 error of rint(32 x + 32.5)
-// in fp32, so a value next to an edge gets the same count in either cell.
-struct NF4Cell {
-  float thr;
-  uint32_t base;
+// from a cell edge, far more than any rounding of x next to an edge, so a
+// value there gets the same count in either cell.  33 entries of 4 bytes
+// fit the 32 shared-memory banks with only cells 0 and 32 (x = -1, x = 1)
+// sharing one.
+constexpr int kNF4Cells = 33;
+struct NF4CellTable {
+  float thr[kNF4Cells];
+  uint32_t base[kNF4Cells];
 };
-struct NF4Cells {
-  NF4Cell c[66];
-};
-constexpr NF4Cells make_nf4_cells() {
-  NF4Cells t{};
-  for (int i = 0; i < 66; ++i) {
-    const float lo = static_cast<float>(i - 33) / 32.0f, hi = static_cast<float>(i - 32) / 32.0f;
+constexpr float nf4_cell_lo(int i) { return static_cast<float>(2 * i - 33) / 32.0f; }
+constexpr float nf4_cell_hi(int i) { return static_cast<float>(2 * i - 31) / 32.0f; }
+constexpr NF4CellTable make_nf4_cells() {
+  NF4CellTable t{};
+  for (int i = 0; i < kNF4Cells; ++i) {
     uint32_t base = 0;
     float thr = 2.0f;
     for (int j = 0; j < 15; ++j) {
-      if (kNF4Threshold[j] < lo) ++base;
-      else if (kNF4Threshold[j] < hi && thr == 2.0f) thr = kNF4Threshold[j];
+      if (kNF4Threshold[j] < nf4_cell_lo(i)) ++base;
+      else if (kNF4Threshold[j] < nf4_cell_hi(i) && thr == 2.0f) thr = kNF4Threshold[j];
     }
-    t.c[i] = NF4Cell{thr, base};
+    t.thr[i] = thr;
+    t.base[i] = base;
   }
   return t;
 }
-constexpr NF4Cells kNF4Cells = make_nf4_cells();
+constexpr NF4CellTable kNF4CellTable = make_nf4_cells();
 constexpr bool nf4_cells_ok() {
-  for (int i = 0; i < 66; ++i) {
-    const float lo = static_cast<float>(i - 33) / 32.0f, hi = static_cast<float>(i - 32) / 32.0f;
+  for (int i = 0; i < kNF4Cells; ++i) {
     int inside = 0;
     for (int j = 0; j < 15; ++j) {
-      if (kNF4Threshold[j] >= lo && kNF4Threshold[j] < hi) ++inside;
-      const float d1 = kNF4Threshold[j] - lo, d2 = kNF4Threshold[j] - hi;
+      if (kNF4Threshold[j] >= nf4_cell_lo(i) && kNF4Threshold[j] < nf4_cell_hi(i)) ++inside;
+      const float d1 = kNF4Threshold[j] - nf4_cell_lo(i), d2 = kNF4Threshold[j] - nf4_cell_hi(i);
       if ((d1 < 1e-5f && d1 > -1e-5f) || (d2 < 1e-5f && d2 > -1e-5f)) return false;   // too near an edge
     }
     if (inside > 1) return false;
   }
-  return kNF4Cells.c[0].base == 0 && kNF4Cells.c[65].base == 15 && kNF4Cells.c[33].base == 7;
+  return kNF4CellTable.base[0] == 0 && kNF4CellTable.base[32] == 15 && kNF4CellTable.base[16] == 7 &&
+         kNF4CellTable.thr[0] == 2.0f && kNF4CellTable.thr[32] == 2.0f;
 }
 static_assert(nf4_cells_ok(), "NF4 encoder cell table");
-__constant__ NF4Cells c_nf4_cells = kNF4Cells;
+__constant__ NF4CellTable c_nf4_cells = kNF4CellTable;
 
 // every entry present (a lost initializer would silently read as 0)
 static_assert(kNF4Level[0] == -1.0f && kNF4Level[7] == 0.0f && kNF4Level[15] == 1.0f, "NF4 levels");

@@ -147,9 +147,10 @@ def _sweep_blocks(absmax: float, centres, half_width: int) -> np.ndarray:
 
 
 def test_encoder_cells_and_thresholds_swept_binary32():
-    # The kernel counts #{i : x > t_i} through a table of 66 cells of width
-    # 1/32 (one compare per cell).  Sweep every binary32 within 1500 ulps of
-    # each of the 15 thresholds and each of the 65 cell edges j/32, at
+    # The kernel counts #{i : x > t_i} through a table of 33 cells of width
+    # 1/16 (one compare per cell; edges at the odd multiples of 1/32).  Sweep
+    # every binary32 within 1500 ulps of each of the 15 thresholds and of
+    # every multiple of 1/32 in [-1, 1] (the edges and the cell centres), at
     # absmax values that are powers of two (x = w / absmax exactly) and not,
     # and require the codes, scales and dequantised weights bit for bit.
     lv = O.nf4_levels().astype(np.float64)
