@@ -49,7 +49,11 @@
 
 namespace qlora {
 
-constexpr int kPairRingA = 6;                    // activation ring depth
+// MSUB = 1: one 256-row M tile per pair; MSUB = 2: two (a 512 x 256 output
+// tile), so every dequantised weight stage feeds 512 tokens.
+template <int MSUB> struct PairRing;
+template <> struct PairRing<1> { static constexpr int A = 6; };   // activation ring depth
+template <> struct PairRing<2> { static constexpr int A = 3; };
 constexpr int kPairRingC = 6;                    // packed-code ring depth
 constexpr int kPairRingW = 6;                    // dequantised-weight ring depth
 constexpr int kPairDeqGroups = 3;                // group it % 3 decodes stage it (owns W slots g, g + 3)
@@ -61,7 +65,9 @@ static_assert(kPairRingW % kPairDeqGroups == 0, "each weight slot must belong to
 static_assert(kPairRingC % kPairDeqGroups == 0, "each code slot must belong to one dequant group");
 constexpr int kPairDeqWarps = 4;                 // warps per group (128 weight rows)
 constexpr int kPairIssuers = 2;
-static_assert(kPairRingA % kPairIssuers == 0 && kPairRingW % kPairIssuers == 0, "each operand slot must belong to one issuer");
+// with MSUB = 1 the issuers alternate stages (G = 2); with MSUB = 2 each
+// takes every stage (G = 1)
+static_assert(PairRing<1>::A % kPairIssuers == 0 && kPairRingW % kPairIssuers == 0, "each operand slot must belong to one issuer");
 constexpr int kPairIssuerWarp1 = 2 + kPairDeqGroups * kPairDeqWarps;   // second MMA issuer
 // The code producer has a warp of its own: as a second lane of the
 // activation producer's warp it was starved while lane 0 spun on its ring
@@ -69,24 +75,29 @@ constexpr int kPairIssuerWarp1 = 2 + kPairDeqGroups * kPairDeqWarps;   // second
 // stage ahead instead of a whole ring ahead.
 constexpr int kPairCodesWarp = kPairIssuerWarp1 + 1;
 constexpr int kPairThreads = 32 * (kPairCodesWarp + 1);
-constexpr uint32_t kPairABytes = 128 * 64 * 2;   // 16 KB activations (this CTA's half)
+constexpr uint32_t kPairABytes = 128 * 64 * 2;   // 16 KB activations (this CTA's half of one M tile)
 constexpr uint32_t kPairWBytes = 128 * 64 * 2;   // 16 KB dequantised weight half
 constexpr uint32_t kPairCBytes = 128 * 64 / 2;   //  4 KB packed codes
-constexpr uint32_t kPairOffW = kPairRingA * kPairABytes;
+// the activation ring is 96 KB for either MSUB (6 x 16 KB or 3 x 32 KB)
+static_assert(PairRing<1>::A * kPairABytes == PairRing<2>::A * 2 * kPairABytes, "same layout for both MSUB");
+constexpr uint32_t kPairOffW = PairRing<1>::A * kPairABytes;
 constexpr uint32_t kPairOffC = kPairOffW + kPairRingW * kPairWBytes;
 constexpr uint32_t kPairOffBar = kPairOffC + kPairRingC * kPairCBytes;
 constexpr uint32_t kPairSmemBytes = kPairOffBar + 1024 /*align*/ + 512 /*bars*/ + 4 * kPairDeqGroups * 128;
-constexpr uint32_t kPairTmemCols = 512;   // D0 (even stages) at 0, D1 (odd stages) at 256
+constexpr uint32_t kPairTmemCols = 512;   // two 256-column accumulators
 static_assert(kPairSmemBytes <= 227 * 1024, "pair kernel shared memory");
 
-template <int MODE, bool WDENSE = false>
+template <int MODE, bool WDENSE = false, int MSUB = 1>
 __global__ void __launch_bounds__(kPairThreads, 1)
     k_gemm_nf4_pair(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                     const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
                     const GemmArgs args) {
+  static_assert(MSUB == 1 || MSUB == 2, "one or two M tiles per pair");
+  constexpr int kPairRingA = PairRing<MSUB>::A;
+  constexpr uint32_t kSlotA = MSUB * kPairABytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  auto slot_a = [&](int it) { return base + (it % kPairRingA) * kPairABytes; };
+  auto slot_a = [&](int it) { return base + (it % kPairRingA) * kSlotA; };
   auto slot_w = [&](int it) { return base + kPairOffW + (it % kPairRingW) * kPairWBytes; };
   auto slot_c = [&](int it) { return base + kPairOffC + (it % kPairRingC) * kPairCBytes; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + kPairOffBar);
@@ -105,7 +116,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * 256 + rank * 128;   // this CTA's activation rows
+  // this CTA's activation rows: m0 + 256 s .. + 127 for M tile s < MSUB
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * 256 * MSUB + rank * 128;
   const int64_t np0 = static_cast<int64_t>(blockIdx.x >> 1) * 256;           // pair's output columns
   const int64_t nc0 = np0 + rank * 128;                                      // this CTA's B half
   const int nl1 = (args.lora_r16 + 63) / 64;
@@ -113,14 +125,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int total = args.num_kt + num_lt;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPairRingA; ++i) { mbar_init(smem_u32(&full_a[i]), 1); mbar_init(smem_u32(&empty_a[i]), 1); }
+    // MSUB = 2: both issuers read every stage, so each slot is freed by two commits
+    for (int i = 0; i < kPairRingA; ++i) { mbar_init(smem_u32(&full_a[i]), 1); mbar_init(smem_u32(&empty_a[i]), MSUB); }
     for (int i = 0; i < kPairRingC; ++i) {
       mbar_init(smem_u32(&full_c[i]), 1);
       mbar_init(smem_u32(&empty_c[i]), kPairDeqWarps);
     }
     for (int i = 0; i < kPairRingW; ++i) {
       mbar_init(smem_u32(&full_w[i]), 2 * kPairDeqWarps);
-      mbar_init(smem_u32(&empty_w[i]), 1);
+      mbar_init(smem_u32(&empty_w[i]), MSUB);
     }
     mbar_init(smem_u32(acc_full), kPairIssuers);
     *abort_flag = 0;
@@ -153,8 +166,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           break;
         const uint32_t fa = leader_bar(&full_a[ia]);
         if (it < args.num_kt) {
-          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * kPairABytes);
-          tma_load_2d_pair(smem_u32(slot_a(it)), &tm_act, fa, it * 64, static_cast<int32_t>(m0));
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * kSlotA);
+#pragma unroll
+          for (int t = 0; t < MSUB; ++t)
+            tma_load_2d_pair(smem_u32(slot_a(it)) + t * kPairABytes, &tm_act, fa, it * 64, static_cast<int32_t>(m0 + 256 * t));
         } else {
           // adapter stage: the A tile here; the adapter B tile is loaded into
           // the weight slot, and its bytes counted on that slot's full_w, by
@@ -165,8 +180,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const int lt = it - args.num_kt;
           const int li = lt % nl1;
           const int64_t arow = (lt / nl1) * args.lora_lo_row + m0;
-          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * kPairABytes);
-          tma_load_2d_pair(smem_u32(slot_a(it)), &tm_la, fa, li * 64, static_cast<int32_t>(arow));
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * kSlotA);
+#pragma unroll
+          for (int t = 0; t < MSUB; ++t)
+            tma_load_2d_pair(smem_u32(slot_a(it)) + t * kPairABytes, &tm_la, fa, li * 64, static_cast<int32_t>(arow + 256 * t));
         }
         ++issued;
       }
@@ -210,22 +227,27 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   } else if (warp == 1 || warp == kPairIssuerWarp1) {
     // ------------------------------------------------- MMA issuers (leader)
     if (leader && lane == 0) {
+      // MSUB = 1: issuer i takes the stages it = i (mod 2) into D_i (summed
+      // in the epilogue); MSUB = 2: issuer i takes every stage for M tile i
+      // into D_i
       const int me = (warp == 1) ? 0 : 1;
       const uint32_t dcol = tmem_d + 256u * me;
+      const int first = (MSUB == 1) ? me : 0;
+      constexpr int step = (MSUB == 1) ? kPairIssuers : 1;
       constexpr uint32_t idesc = idesc_bf16(256, 256, 0, MODE == kModeDx ? 1 : 0);
-      for (int it = me; it < total; it += kPairIssuers) {
+      for (int it = first; it < total; it += step) {
         const int ia = it % kPairRingA, iw = it % kPairRingW;
         if (!mbar_wait(smem_u32(&full_a[ia]), par(it, kPairRingA), abort_flag, args.status)) break;
         if (!mbar_wait(smem_u32(&full_w[iw]), par(it, kPairRingW), abort_flag, args.status)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(slot_a(it));
+        const uint32_t a_base = smem_u32(slot_a(it)) + (MSUB == 1 ? 0u : me * kPairABytes);
         const uint32_t w_base = smem_u32(slot_w(it));
         const int nk = (it < args.num_kt) ? 4 : min(4, (args.lora_r16 - ((it - args.num_kt) % nl1) * 64) / 16);
         for (int k = 0; k < nk; ++k) {
           const uint64_t adesc = sw128_desc(a_base + k * 32, 16, 1024);
           const uint64_t bdesc = (MODE == kModeFwd) ? sw128_desc(w_base + k * 32, 16, 1024)
                                                     : sw128_desc(w_base + k * 2048, 8192, 1024);
-          umma_bf16_pair(dcol, adesc, bdesc, idesc, (it > me || k > 0) ? 1u : 0u);
+          umma_bf16_pair(dcol, adesc, bdesc, idesc, (it > first || k > 0) ? 1u : 0u);
         }
         umma_commit_pair(smem_u32(&empty_a[ia]), 0x3);
         umma_commit_pair(smem_u32(&empty_w[iw]), 0x3);
@@ -360,19 +382,38 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     tc_fence_after();
     if (!*abort_flag) {
       const int q = warp & 3;
-      const int64_t row = m0 + q * 32 + lane;
       const uint32_t taddr = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
+      if (MSUB == 1) {
+        // D_0 + D_1 (fixed order); with a single stage the second issuer had
+        // none and D_1 was never written
+        const int64_t row = m0 + q * 32 + lane;
+        const bool two = total > 1;
 #pragma unroll 1
-      for (int c = g; c < 16; c += kPairDeqGroups) {
-        const int col = c * 16;
-        uint32_t r[16], r1[16];
-        tmem_ld16(taddr + col, r);
-        tmem_ld16(taddr + 256 + col, r1);
-        tmem_ld_wait();
+        for (int c = g; c < 16; c += kPairDeqGroups) {
+          const int col = c * 16;
+          uint32_t r[16], r1[16];
+          tmem_ld16(taddr + col, r);
+          tmem_ld16(taddr + 256 + col, r1);
+          tmem_ld_wait();
+          if (two) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r1[i]));
-        const int64_t gc = np0 + col;
-        if (row < args.M && gc < args.out_cols) gemm_store16(args, row, gc, r);
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r1[i]));
+          }
+          const int64_t gc = np0 + col;
+          if (row < args.M && gc < args.out_cols) gemm_store16(args, row, gc, r);
+        }
+      } else {
+        // D_t holds M tile t
+#pragma unroll 1
+        for (int u = g; u < 32; u += kPairDeqGroups) {
+          const int t = u >> 4, col = (u & 15) * 16;
+          const int64_t row = m0 + 256 * t + q * 32 + lane;
+          uint32_t r[16];
+          tmem_ld16(taddr + 256 * t + col, r);
+          tmem_ld_wait();
+          const int64_t gc = np0 + col;
+          if (row < args.M && gc < args.out_cols) gemm_store16(args, row, gc, r);
+        }
       }
     }
   }

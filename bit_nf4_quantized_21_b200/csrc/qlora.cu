@@ -87,10 +87,13 @@ bool ensure_smem_attrs() {
   const int max_smem = 227 * 1024;
   bool ok = cudaFuncSetAttribute(k_gemm_nf4<kModeFwd>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_gemm_nf4<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeFwd>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeDx>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeFwd, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(k_gemm_nf4_pair<kModeDx, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
+  const void* pair_kernels[] = {
+      reinterpret_cast<const void*>(k_gemm_nf4_pair<kModeFwd, false, 1>), reinterpret_cast<const void*>(k_gemm_nf4_pair<kModeDx, false, 1>),
+      reinterpret_cast<const void*>(k_gemm_nf4_pair<kModeFwd, true, 1>), reinterpret_cast<const void*>(k_gemm_nf4_pair<kModeDx, true, 1>),
+      reinterpret_cast<const void*>(k_gemm_nf4_pair<kModeFwd, false, 2>), reinterpret_cast<const void*>(k_gemm_nf4_pair<kModeDx, false, 2>),
+      reinterpret_cast<const void*>(k_gemm_nf4_pair<kModeFwd, true, 2>), reinterpret_cast<const void*>(k_gemm_nf4_pair<kModeDx, true, 2>)};
+  for (const void* k : pair_kernels)
+    ok = ok && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_skinny<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) == cudaSuccess;
@@ -110,6 +113,26 @@ int sm_count() {
     cache[dev].store(v);
   }
   return v;
+}
+
+// M tiles per pair launch of the fused GEMM: 1 (256 rows) or 2 (512 rows).
+// Two tiles feed every dequantised weight stage to 512 tokens, which halves
+// the decode work per flop; one tile gives twice as many pair tiles, which
+// packs better into the pairs of SMs when the grid is a few waves.  The
+// estimate takes a 512-row tile at kPair2Cost / 10 of a 256-row tile's
+// time (both decode the same weights; the larger does twice the MMAs):
+// 1.5-1.6 measured on B200 over the LLaMA-7B and 65B projection shapes.
+// qlora_debug_set_pair_mtiles can force either (0 = this choice).
+std::atomic<int> g_force_mtiles{0};
+constexpr int64_t kPair2Cost = 16;
+int pair_mtiles(int64_t M, int64_t out_cols) {
+  const int f = g_force_mtiles.load();
+  if (f == 1 || f == 2) return f;
+  if (M <= 256) return 1;
+  const int64_t pairs = std::max<int64_t>(1, sm_count() / 2);
+  const int64_t nt = cdiv(out_cols, 256);
+  const int64_t w1 = cdiv(nt * cdiv(M, 256), pairs), w2 = cdiv(nt * cdiv(M, 512), pairs);
+  return (w2 * kPair2Cost < w1 * 10) ? 2 : 1;
 }
 
 // Record a caller's timing event on the stream.  Under stream capture the
@@ -416,7 +439,8 @@ qlora_status launch_gemm(int mode, const CUtensorMap& tact, const CUtensorMap& t
 
 
 // Fused NF4 GEMM of one call: tensor maps + dispatch.  M > 128 takes the
-// 2-SM pair kernel (256 x 256 tiles per pair), smaller M the 1-CTA kernel.
+// 2-SM pair kernel (256 x 256 or 512 x 256 tiles per pair, pair_mtiles),
+// smaller M the 1-CTA kernel.
 //   fwd: act = X [M, K], la = s*T planes [2M, r8], lb = B [N, r8], out Y [M, N]
 //   dX : act = dY [M, N], la = s*G planes [2M, r8], lb = A [r, K], out dX [M, K]
 // The fused GEMM of the forward (mode kModeFwd) or of dX (kModeDx), over
@@ -471,8 +495,9 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
 
   if (ev && ev->gemm_start && record_event(static_cast<cudaEvent_t>(ev->gemm_start), cs) != cudaSuccess)
     return QLORA_ERR_CUDA;
+  const int mt = pair_mtiles(d.M, a.out_cols);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * cdiv(a.out_cols, 256)), static_cast<unsigned>(cdiv(d.M, 256)));
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * cdiv(a.out_cols, 256)), static_cast<unsigned>(cdiv(d.M, 256 * mt)));
   cfg.blockDim = dim3(kPairThreads);
   cfg.dynamicSmemBytes = kPairSmemBytes;
   cfg.stream = cs;
@@ -484,12 +509,21 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (dense)
-    e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, true>, tact, tcodes, tla, tlb, a)
-            : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, true>, tact, tcodes, tla, tlb, a);
-  else
-    e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd>, tact, tcodes, tla, tlb, a)
-            : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx>, tact, tcodes, tla, tlb, a);
+  if (mt == 2) {
+    if (dense)
+      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, true, 2>, tact, tcodes, tla, tlb, a)
+              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, true, 2>, tact, tcodes, tla, tlb, a);
+    else
+      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, false, 2>, tact, tcodes, tla, tlb, a)
+              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, false, 2>, tact, tcodes, tla, tlb, a);
+  } else {
+    if (dense)
+      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, true, 1>, tact, tcodes, tla, tlb, a)
+              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, true, 1>, tact, tcodes, tla, tlb, a);
+    else
+      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, false, 1>, tact, tcodes, tla, tlb, a)
+              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, false, 1>, tact, tcodes, tla, tlb, a);
+  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     return QLORA_ERR_CUDA;
@@ -950,6 +984,12 @@ qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16
 qlora_status qlora_debug_set_wait_limit(uint64_t ns) {
   const unsigned long long v = ns ? static_cast<unsigned long long>(ns) : QLORA_WAIT_NS;
   return cudaMemcpyToSymbol(g_qlora_wait_ns, &v, sizeof(v)) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_debug_set_pair_mtiles(int n) {
+  if (n < 0 || n > 2) return QLORA_ERR_INVALID_ARG;
+  g_force_mtiles.store(n);
+  return QLORA_OK;
 }
 
 qlora_status qlora_debug_inject_stall(int on) {

@@ -31,6 +31,7 @@ EXPORTED = (
     "qlora_adam_step", "qlora_merge_nf4", "qlora_workspace_bytes_dropout", "qlora_lora_dropout_mask",
     "qlora_linear_fwd_dropout", "qlora_linear_bwd_dropout", "qlora_paged_alloc", "qlora_paged_free",
     "qlora_paged_prefetch", "qlora_debug_set_wait_limit", "qlora_debug_inject_stall",
+    "qlora_debug_set_pair_mtiles",
 )
 
 
@@ -130,6 +131,8 @@ def lib() -> ctypes.CDLL:
             L.qlora_debug_set_wait_limit.restype = I32
             L.qlora_debug_inject_stall.argtypes = [I32]
             L.qlora_debug_inject_stall.restype = I32
+            L.qlora_debug_set_pair_mtiles.argtypes = [I32]
+            L.qlora_debug_set_pair_mtiles.restype = I32
             L.qlora_status_string.argtypes = [I32]
             L.qlora_status_string.restype = ctypes.c_char_p
             L.qlora_version.argtypes = []

@@ -341,10 +341,20 @@ qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16
  *     runs out; the launch then ends early with the timeout bit set and the
  *     call's outputs unspecified.  Calls after it is switched off are
  *     unaffected (each call clears the arrival counters it uses).
- * Neither is for production use; both apply to kernels enqueued afterwards.
+ *   qlora_debug_set_pair_mtiles(n): the fused GEMM for M > 128 runs on
+ *     pairs of SMs with n = 1 (256 x 256) or n = 2 (512 x 256) output tiles
+ *     per pair; 0 (the default) lets each call choose from its shape, 1 or
+ *     2 forces that tile for every later call of this process (so that
+ *     tests reach both); other values return QLORA_ERR_INVALID_ARG.  Both
+ *     form the same products; the fp32 accumulation order differs (one
+ *     tile: even and odd 64-deep stages in two accumulators added at the
+ *     end; two tiles: one accumulator per tile), so the last bits of a
+ *     result may differ between the two.
+ * None is for production use; they apply to kernels enqueued afterwards.
  */
 qlora_status qlora_debug_set_wait_limit(uint64_t ns);
 qlora_status qlora_debug_inject_stall(int on);
+qlora_status qlora_debug_set_pair_mtiles(int n);
 
 /*
  * Paged optimiser state ("QLoRA", learning-llms page, the paragraph on paged

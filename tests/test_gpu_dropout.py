@@ -37,6 +37,7 @@ def _nan(shape, dt):
 @pytest.mark.parametrize("M,N,K,r,p", [
     (256, 512, 1024, 16, 0.05),   # the pages' rate, the fused 2-SM GEMM path
     (200, 264, 576, 8, 0.3),      # ragged tiles in every dimension, a higher rate
+    (300, 64, 576, 8, 0.05),      # N = 64: the dX GEMM (adapter not folded) has a single stage
     (96, 136, 448, 5, 0.05),      # 16 < M <= 128: the 1-CTA GEMM; r not a multiple of 8
     (16, 1024, 2048, 16, 0.05),   # decode shape: T inside the weight-streaming kernel
     (1, 8192, 8192, 8, 0.2),      # a single token (8192 outputs in Y and in dX)

@@ -94,6 +94,33 @@ def test_ragged_and_edge_shapes(M, N, K, r):
     _compare(_run(*args, alpha), _oracle(*args, alpha), grad_tol=1e-4)
 
 
+@pytest.mark.parametrize("mtiles", [1, 2])
+@pytest.mark.parametrize("M,N,K,r", [
+    (600, 264, 576, 8),      # two 512-row tiles, the second ragged; N, K ragged
+    (1100, 512, 1024, 16),   # three 512-row tiles, the last with 76 rows
+    (300, 320, 64, 5),       # one 64-deep weight stage; r not a multiple of 8
+    (520, 136, 448, 64),     # 8 rows in the second 512-row tile
+])
+def test_pair_one_and_two_m_tiles(mtiles, M, N, K, r):
+    # the 2-SM GEMM (M > 128) with one 256-row or two 256-row M tiles per
+    # pair, forced for forward and dX alike
+    L = q.lib()
+    assert L.qlora_debug_set_pair_mtiles(mtiles) == 0
+    try:
+        args = _problem(M, N, K, r, seed=3 * M + N + K + r + mtiles)
+        alpha = 2.0 * r
+        _compare(_run(*args, alpha), _oracle(*args, alpha), grad_tol=1e-4)
+    finally:
+        assert L.qlora_debug_set_pair_mtiles(0) == 0
+
+
+def test_pair_m_tiles_hook_rejects_bad_values():
+    L = q.lib()
+    assert L.qlora_debug_set_pair_mtiles(3) != 0
+    assert L.qlora_debug_set_pair_mtiles(-1) != 0
+    assert L.qlora_debug_set_pair_mtiles(0) == 0
+
+
 @pytest.mark.parametrize("proj", [0, 4, 6])   # q 4096x4096, gate 11008x4096, down 4096x11008
 def test_llama7b_projection_full(proj):
     wl = inputs.LLAMA7B
