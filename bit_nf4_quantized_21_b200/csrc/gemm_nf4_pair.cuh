@@ -10,7 +10,8 @@
 //   (MMA B half), and TMEM rows for its 128 activation rows x 256 columns.
 //
 // Three shared-memory rings per CTA; stage `it` (64 deep) uses slot
-// it % depth of each:
+// it % depth of each (depths for one M tile per pair; with two, the
+// activation slots hold both tiles' halves, PairRing below):
 //   activations  6 x 16 KB  pair TMA by the producer warp (0), completing on
 //                           the leader's full_a; freed by the MMA (empty_a)
 //   codes        6 x  4 KB  local TMA by the code warp (15) (full_c); a
@@ -50,24 +51,26 @@
 namespace qlora {
 
 // MSUB = 1: one 256-row M tile per pair; MSUB = 2: two (a 512 x 256 output
-// tile), so every dequantised weight stage feeds 512 tokens.
+// tile), so every dequantised weight stage feeds 512 tokens.  Ring depths
+// per MSUB (activation slots hold MSUB x 16 KB per CTA).
 template <int MSUB> struct PairRing;
-template <> struct PairRing<1> { static constexpr int A = 6; };   // activation ring depth
-template <> struct PairRing<2> { static constexpr int A = 3; };
+template <> struct PairRing<1> { static constexpr int A = 6, W = 6; };
+template <> struct PairRing<2> { static constexpr int A = 3, W = 6; };
 constexpr int kPairRingC = 6;                    // packed-code ring depth
-constexpr int kPairRingW = 6;                    // dequantised-weight ring depth
-constexpr int kPairDeqGroups = 3;                // group it % 3 decodes stage it (owns W slots g, g + 3)
+constexpr int kPairDeqGroups = 3;                // group it % 3 decodes stage it (owns W slots it % depth)
 // A waiter that takes every G-th stage must own whole slots: with a ring
 // depth that is not a multiple of G it could come to a slot whose previous
 // phase (another waiter's stage) is still pending, and a parity wait would
 // then take the phase before that for the one it wants.
-static_assert(kPairRingW % kPairDeqGroups == 0, "each weight slot must belong to one dequant group");
+static_assert(PairRing<1>::W % kPairDeqGroups == 0 && PairRing<2>::W % kPairDeqGroups == 0,
+              "each weight slot must belong to one dequant group");
 static_assert(kPairRingC % kPairDeqGroups == 0, "each code slot must belong to one dequant group");
 constexpr int kPairDeqWarps = 4;                 // warps per group (128 weight rows)
 constexpr int kPairIssuers = 2;
 // with MSUB = 1 the issuers alternate stages (G = 2); with MSUB = 2 each
 // takes every stage (G = 1)
-static_assert(PairRing<1>::A % kPairIssuers == 0 && kPairRingW % kPairIssuers == 0, "each operand slot must belong to one issuer");
+static_assert(PairRing<1>::A % kPairIssuers == 0 && PairRing<1>::W % kPairIssuers == 0,
+              "each operand slot must belong to one issuer");
 constexpr int kPairIssuerWarp1 = 2 + kPairDeqGroups * kPairDeqWarps;   // second MMA issuer
 // The code producer has a warp of its own: as a second lane of the
 // activation producer's warp it was starved while lane 0 spun on its ring
@@ -78,12 +81,13 @@ constexpr int kPairThreads = 32 * (kPairCodesWarp + 1);
 constexpr uint32_t kPairABytes = 128 * 64 * 2;   // 16 KB activations (this CTA's half of one M tile)
 constexpr uint32_t kPairWBytes = 128 * 64 * 2;   // 16 KB dequantised weight half
 constexpr uint32_t kPairCBytes = 128 * 64 / 2;   //  4 KB packed codes
-// the activation ring is 96 KB for either MSUB (6 x 16 KB or 3 x 32 KB)
-static_assert(PairRing<1>::A * kPairABytes == PairRing<2>::A * 2 * kPairABytes, "same layout for both MSUB");
-constexpr uint32_t kPairOffW = PairRing<1>::A * kPairABytes;
-constexpr uint32_t kPairOffC = kPairOffW + kPairRingW * kPairWBytes;
-constexpr uint32_t kPairOffBar = kPairOffC + kPairRingC * kPairCBytes;
-constexpr uint32_t kPairSmemBytes = kPairOffBar + 1024 /*align*/ + 512 /*bars*/ + 4 * kPairDeqGroups * 128;
+template <int MSUB> struct PairLayout {
+  static constexpr uint32_t OffW = PairRing<MSUB>::A * MSUB * kPairABytes;
+  static constexpr uint32_t OffC = OffW + PairRing<MSUB>::W * kPairWBytes;
+  static constexpr uint32_t OffBar = OffC + kPairRingC * kPairCBytes;
+  static constexpr uint32_t Bytes = OffBar + 1024 /*align*/ + 512 /*bars*/;
+};
+constexpr uint32_t kPairSmemBytes = PairLayout<1>::Bytes > PairLayout<2>::Bytes ? PairLayout<1>::Bytes : PairLayout<2>::Bytes;
 constexpr uint32_t kPairTmemCols = 512;   // two 256-column accumulators
 static_assert(kPairSmemBytes <= 227 * 1024, "pair kernel shared memory");
 
@@ -94,13 +98,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const GemmArgs args) {
   static_assert(MSUB == 1 || MSUB == 2, "one or two M tiles per pair");
   constexpr int kPairRingA = PairRing<MSUB>::A;
+  constexpr int kPairRingW = PairRing<MSUB>::W;
   constexpr uint32_t kSlotA = MSUB * kPairABytes;
+  using Lay = PairLayout<MSUB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   auto slot_a = [&](int it) { return base + (it % kPairRingA) * kSlotA; };
-  auto slot_w = [&](int it) { return base + kPairOffW + (it % kPairRingW) * kPairWBytes; };
-  auto slot_c = [&](int it) { return base + kPairOffC + (it % kPairRingC) * kPairCBytes; };
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kPairOffBar);
+  auto slot_w = [&](int it) { return base + Lay::OffW + (it % kPairRingW) * kPairWBytes; };
+  auto slot_c = [&](int it) { return base + Lay::OffC + (it % kPairRingC) * kPairCBytes; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + Lay::OffBar);
   uint64_t* full_a = bars;                                  // [A] leader: activation halves (+ adapter tiles)
   uint64_t* empty_a = full_a + kPairRingA;                  // [A] local: MMA done with the activations
   uint64_t* full_c = empty_a + kPairRingA;                  // [C] local: codes landed
