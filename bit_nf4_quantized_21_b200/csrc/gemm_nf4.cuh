@@ -63,6 +63,7 @@ struct GemmArgs {
   int lora_r16;          // adapter rank rounded up to 16 (0: no adapter)
   int64_t lora_lo_row;   // row of the adapter operand where the lo plane starts (= M)
   int* status;
+  int tma_out;           // 2-SM kernel: 1 when its tm_out maps `out` (bf16, 64 x 32 boxes, 128-byte swizzle)
 };
 
 // Output columns [gc, gc + 16) of row `row` (fp32 accumulator words r):

@@ -10,8 +10,9 @@
 //   (MMA B half), and TMEM rows for its 128 activation rows x 256 columns.
 //
 // Three shared-memory rings per CTA; stage `it` (64 deep) uses slot
-// it % depth of each (depths for one M tile per pair; with two, the
-// activation slots hold both tiles' halves, PairRing below):
+// it % depth of each (depths for one M tile per pair; with two, 4
+// activation slots hold both tiles' halves and there are 3 weight slots,
+// PairRing below):
 //   activations  6 x 16 KB  pair TMA by the producer warp (0), completing on
 //                           the leader's full_a; freed by the MMA (empty_a)
 //   codes        6 x  4 KB  local TMA by the code warp (15) (full_c); a
@@ -37,7 +38,8 @@
 // takes every G-th stage (issuers G = 2, dequant groups G = 3) owns whole
 // slots because each ring depth is a multiple of its waiters' G, so no
 // waiter can be two phases behind and the 1-bit phase parity is safe.
-// Epilogue: every CTA reads its own TMEM half (tcgen05.ld) and writes bf16.
+// Epilogue: all 16 warps of every CTA read its own TMEM half (tcgen05.ld)
+// and write bf16.
 //
 // WDENSE = true is the same GEMM over a dense bf16 weight (plain LoRA, the
 // baseline the QLoRA pages compare against): the weight tile of every
@@ -55,7 +57,7 @@ namespace qlora {
 // per MSUB (activation slots hold MSUB x 16 KB per CTA).
 template <int MSUB> struct PairRing;
 template <> struct PairRing<1> { static constexpr int A = 6, W = 6; };
-template <> struct PairRing<2> { static constexpr int A = 3, W = 6; };
+template <> struct PairRing<2> { static constexpr int A = 4, W = 3; };
 constexpr int kPairRingC = 6;                    // packed-code ring depth
 constexpr int kPairDeqGroups = 3;                // group it % 3 decodes stage it (owns W slots it % depth)
 // A waiter that takes every G-th stage must own whole slots: with a ring
@@ -95,7 +97,7 @@ template <int MODE, bool WDENSE = false, int MSUB = 1>
 __global__ void __launch_bounds__(kPairThreads, 1)
     k_gemm_nf4_pair(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                     const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
-                    const GemmArgs args) {
+                    const __grid_constant__ CUtensorMap tm_out, const GemmArgs args) {
   static_assert(MSUB == 1 || MSUB == 2, "one or two M tiles per pair");
   constexpr int kPairRingA = PairRing<MSUB>::A;
   constexpr int kPairRingW = PairRing<MSUB>::W;
@@ -371,63 +373,119 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const uint64_t t0 = global_ns();
       while (global_ns() - t0 < 1000000ull) {}
     }
+  }
 
-    // ------------------------------------------------------------ epilogue
-    {
-      const uint32_t bar = smem_u32(acc_full);
-      const uint64_t t0 = global_ns(), limit = qlora_wait_limit();
-      bool ok = true;
-      while (!mbar_try_wait_cluster(bar, 0)) {
-        if (global_ns() - t0 > limit) { ok = false; break; }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        if (args.status) atomicOr(args.status, QLORA_DEV_TIMEOUT);
-      }
+  // ------------------------------------------------------------ epilogue
+  // Every warp, the role warps included: warp w reads TMEM lanes 32 (w % 4)
+  // .. + 31 (its quarter of the accumulator rows) and takes a quarter of
+  // the 16-column chunks, contiguous; four (one M tile: two pairs of) TMEM
+  // loads go out before each wait.  With a bf16 output the warp stages its
+  // 32 rows x 64 columns per box in shared memory (128-byte swizzle: the
+  // lanes' 16-byte pieces of one column range fall in different banks) and
+  // one lane writes the box with a TMA store, so the global writes are whole
+  // rows of the box instead of 32 scattered 16-byte pieces per instruction.
+  // After the last MMA every ring is free: warp w stages at base + 8 KB w.
+  // Single-lane roles leave their warps diverged, and tcgen05.ld is
+  // warp-collective: reconverge first.
+  __syncwarp();
+  {
+    const uint32_t bar = smem_u32(acc_full);
+    const uint64_t t0 = global_ns(), limit = qlora_wait_limit();
+    bool ok = true;
+    while (!mbar_try_wait_cluster(bar, 0)) {
+      if (global_ns() - t0 > limit) { ok = false; break; }
     }
-    tc_fence_after();
-    if (!*abort_flag) {
-      const int q = warp & 3;
-      const uint32_t taddr = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
-      if (MSUB == 1) {
-        // D_0 + D_1 (fixed order); with a single stage the second issuer had
-        // none and D_1 was never written
-        const int64_t row = m0 + q * 32 + lane;
-        const bool two = total > 1;
+    if (!ok) {
+      *abort_flag = 1;
+      if (args.status) atomicOr(args.status, QLORA_DEV_TIMEOUT);
+    }
+  }
+  __syncwarp();
+  tc_fence_after();
+  if (!*abort_flag) {
+    const int q = warp & 3, j = warp >> 2;
+    const uint32_t taddr = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
+    uint8_t* stg = base + warp * 8192;
+    // columns 16 c .. 16 c + 15 (c < 4) of this lane's row of a 64-column box, as bf16
+    auto stage16 = [&](uint8_t* box, int c, const uint32_t (&r)[16]) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+      uint8_t* row = box + lane * 128;
+      *reinterpret_cast<uint4*>(row + (((2 * c) ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ (lane & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    };
+    // the box at output column x, row y (boxes that start past the edge are skipped; TMA clips the rest)
+    auto store_box = [&](const uint8_t* box, int64_t x, int64_t y) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && x < args.out_cols && y < args.M) {
+        tma_store_2d(&tm_out, smem_u32(box), static_cast<int32_t>(x), static_cast<int32_t>(y));
+        bulk_commit();
+      }
+    };
+    if (MSUB == 1) {
+      // D_0 + D_1 (fixed order); with a single stage the second issuer had
+      // none and D_1 was never written.  Chunks 4j .. 4j + 3 (one box).
+      const int64_t row = m0 + q * 32 + lane;
+      const bool two = total > 1;
 #pragma unroll 1
-        for (int c = g; c < 16; c += kPairDeqGroups) {
-          const int col = c * 16;
-          uint32_t r[16], r1[16];
-          tmem_ld16(taddr + col, r);
-          tmem_ld16(taddr + 256 + col, r1);
-          tmem_ld_wait();
+      for (int i = 0; i < 4; i += 2) {
+        const int col = (4 * j + i) * 16;
+        uint32_t r[2][16], r1[2][16];
+        tmem_ld16(taddr + col, r[0]);
+        tmem_ld16(taddr + 256 + col, r1[0]);
+        tmem_ld16(taddr + col + 16, r[1]);
+        tmem_ld16(taddr + 256 + col + 16, r1[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
           if (two) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r1[i]));
+            for (int e = 0; e < 16; ++e) r[h][e] = __float_as_uint(__uint_as_float(r[h][e]) + __uint_as_float(r1[h][e]));
           }
-          const int64_t gc = np0 + col;
-          if (row < args.M && gc < args.out_cols) gemm_store16(args, row, gc, r);
+          if (args.tma_out) {
+            stage16(stg, i + h, r[h]);
+          } else {
+            const int64_t gc = np0 + col + 16 * h;
+            if (row < args.M && gc < args.out_cols) gemm_store16(args, row, gc, r[h]);
+          }
         }
-      } else {
-        // D_t holds M tile t
+      }
+      if (args.tma_out) store_box(stg, np0 + 64 * j, m0 + q * 32);
+    } else {
+      // D_t holds M tile t.  Chunks 8j .. 8j + 7 (two boxes): warps 0-7
+      // M tile 0, warps 8-15 M tile 1.
+      const int t = j >> 1;
+      const int64_t row = m0 + 256 * t + q * 32 + lane;
 #pragma unroll 1
-        for (int u = g; u < 32; u += kPairDeqGroups) {
-          const int t = u >> 4, col = (u & 15) * 16;
-          const int64_t row = m0 + 256 * t + q * 32 + lane;
-          uint32_t r[16];
-          tmem_ld16(taddr + 256 * t + col, r);
-          tmem_ld_wait();
-          const int64_t gc = np0 + col;
-          if (row < args.M && gc < args.out_cols) gemm_store16(args, row, gc, r);
+      for (int bx = 0; bx < 2; ++bx) {
+        const int col = (j & 1) * 128 + bx * 64;
+        uint32_t r[4][16];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) tmem_ld16(taddr + 256 * t + col + 16 * h, r[h]);
+        tmem_ld_wait();
+        if (args.tma_out) {
+          uint8_t* box = stg + bx * 4096;
+#pragma unroll
+          for (int h = 0; h < 4; ++h) stage16(box, h, r[h]);
+          store_box(box, np0 + col, m0 + 256 * t + q * 32);
+        } else {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int64_t gc = np0 + col + 16 * h;
+            if (row < args.M && gc < args.out_cols) gemm_store16(args, row, gc, r[h]);
+          }
         }
       }
     }
   }
+  // the TMA stores have read their shared-memory boxes (and landed) before the CTA can exit
+  if (args.tma_out && lane == 0) bulk_wait_all();
 
-  // Single-lane roles (producer, MMA issuer) leave their warps diverged;
-  // the CTA/cluster barrier below is warp-aligned, so every warp first
-  // reconverges here -- otherwise the barrier can complete while a lane is
-  // still working and TMEM could be released under it.
+  // The CTA/cluster barrier below is warp-aligned: every warp reconverges
+  // first, so that it cannot complete while a lane is still working and
+  // TMEM be released under it.
   __syncwarp();
   tc_fence_before();
   cluster_sync();   // the peer may still read this CTA's shared memory / arrive on its barriers until here

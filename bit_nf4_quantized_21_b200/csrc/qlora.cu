@@ -492,6 +492,13 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   a.lora_lo_row = d.M;
   a.status = status;
   if (!pair) return launch_gemm(mode, tact, tcodes, tla, tlb, a, ev, cs);
+  // the 2-SM kernel writes a bf16 output with TMA stores (64 x 32 boxes)
+  // when its rows are 16-byte aligned; fp32 output goes out directly
+  CUtensorMap tout = tla;
+  if (!out_f32 && (a.ldo % 8) == 0) {
+    if (bf16_map(&tout, out, a.out_cols, d.M, a.ldo, 64, 32)) a.tma_out = 1;
+    else tout = tla;   // not encodable: direct stores
+  }
 
   if (ev && ev->gemm_start && record_event(static_cast<cudaEvent_t>(ev->gemm_start), cs) != cudaSuccess)
     return QLORA_ERR_CUDA;
@@ -511,18 +518,18 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   cudaError_t e;
   if (mt == 2) {
     if (dense)
-      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, true, 2>, tact, tcodes, tla, tlb, a)
-              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, true, 2>, tact, tcodes, tla, tlb, a);
+      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, true, 2>, tact, tcodes, tla, tlb, tout, a)
+              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, true, 2>, tact, tcodes, tla, tlb, tout, a);
     else
-      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, false, 2>, tact, tcodes, tla, tlb, a)
-              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, false, 2>, tact, tcodes, tla, tlb, a);
+      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, false, 2>, tact, tcodes, tla, tlb, tout, a)
+              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, false, 2>, tact, tcodes, tla, tlb, tout, a);
   } else {
     if (dense)
-      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, true, 1>, tact, tcodes, tla, tlb, a)
-              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, true, 1>, tact, tcodes, tla, tlb, a);
+      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, true, 1>, tact, tcodes, tla, tlb, tout, a)
+              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, true, 1>, tact, tcodes, tla, tlb, tout, a);
     else
-      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, false, 1>, tact, tcodes, tla, tlb, a)
-              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, false, 1>, tact, tcodes, tla, tlb, a);
+      e = fwd ? cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeFwd, false, 1>, tact, tcodes, tla, tlb, tout, a)
+              : cudaLaunchKernelEx(&cfg, k_gemm_nf4_pair<kModeDx, false, 1>, tact, tcodes, tla, tlb, tout, a);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
