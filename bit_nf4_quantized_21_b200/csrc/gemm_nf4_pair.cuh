@@ -185,6 +185,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           // phase of full_w; this thread may be a whole activation ring
           // ahead, and full_a of this slot may still be in an earlier stage's
           // phase, so neither may carry the B tile's bytes)
+          // s*T (s*G) comes from the kernel ahead in the stream
+          if (it == args.num_kt) griddep_wait();
           const int lt = it - args.num_kt;
           const int li = lt % nl1;
           const int64_t arow = (lt / nl1) * args.lora_lo_row + m0;
@@ -325,6 +327,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // tile (rows/columns past the weight's edge arrive as zeros)
         if (((warp - 2) & 3) == 0 && lane == 0) {
           const bool lora = it >= args.num_kt;
+          // the adapter B tile may come from the kernel ahead (the padded B)
+          if (lora && it < args.num_kt + G) griddep_wait();
           const CUtensorMap* map = lora ? &tm_lb : &tm_codes;
           const int32_t kk = lora ? ((it - args.num_kt) % nl1) * 64 : it * 64;
           const uint32_t fw = leader_bar(&full_w[iw]);
@@ -483,6 +487,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   // the TMA stores have read their shared-memory boxes (and landed) before the CTA can exit
   if (args.tma_out && lane == 0) bulk_wait_all();
 
+  // this grid does not complete before the kernel ahead of it (when no
+  // adapter stage waited for it above)
+  if (threadIdx.x == 0) griddep_wait();
   // The CTA/cluster barrier below is warp-aligned: every warp reconverges
   // first, so that it cannot complete while a lane is still working and
   // TMEM be released under it.

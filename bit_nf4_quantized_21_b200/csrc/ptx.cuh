@@ -188,6 +188,18 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // every bulk store this thread committed has completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Programmatic dependent launch.  A kernel launched with programmatic
+// stream serialisation may start before the kernel ahead of it in the
+// stream has finished; griddep_wait blocks the calling thread until that
+// kernel has completed and its memory operations are visible.  The kernel
+// ahead lets its dependents launch once every one of its CTAs has executed
+// griddep_launch_dependents (or exited), so all of its CTAs are resident
+// before any dependent CTA takes a slot.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

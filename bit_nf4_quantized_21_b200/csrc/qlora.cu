@@ -508,13 +508,18 @@ qlora_status run_fused(int mode, const void* act, const qlora_nf4_weight* Wq, co
   cfg.blockDim = dim3(kPairThreads);
   cfg.dynamicSmemBytes = kPairSmemBytes;
   cfg.stream = cs;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the GEMM may start while the adapter
+  // kernel ahead of it (T, or dA + dB in the backward) is still running;
+  // it waits for that kernel only where it reads its results
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e;
   if (mt == 2) {
     if (dense)
@@ -653,23 +658,9 @@ qlora_status linear_bwd_core(const void* dY, const void* X, const Dims& d, const
     st = launch_skinny<0, 1>(j, nullptr, cs);
     if (st != QLORA_OK) return st;
   }
-  // 2. dX = dY W^ + (sG) A; under dropout dY W^ in fp32, then one pass
-  //    adding s ((G A) * keep) / (1 - p) and rounding once
-  if (dX && !drop) {
-    st = run_fused(kModeDx, dY, Wq, Wdense, d, sG, A, dX, events, d_status, cs);
-    if (st != QLORA_OK) return st;
-  } else if (dX) {
-    float* dxf = reinterpret_cast<float*>(ws + WD.dxf);
-    st = run_fused(kModeDx, dY, Wq, Wdense, d, sG, A, dX, events, d_status, cs, dxf, false);
-    if (st != QLORA_OK) return st;
-    k_dropout_dx<<<dropout_grid(d.M * (d.K / 8)), kDropThreads, 0, cs>>>(
-        dxf, reinterpret_cast<const float*>(ws + WD.g32), static_cast<const __nv_bfloat16*>(A), d.M, d.K, d.r,
-        s * inv_q, drop->seed, drop->thr, static_cast<__nv_bfloat16*>(dX));
-    st = check_launch();
-    if (st != QLORA_OK) return st;
-  }
-  // 3. dA = s G^T X (C[k, q] = sum_m X[m, k] Ghl[m, q]) and dB = s dY^T T
-  //    (C[n, q] = sum_m dY[m, n] Thl[m, q]) in one launch
+  // 2. dA = s G^T X (C[k, q] = sum_m X[m, k] Ghl[m, q]) and dB = s dY^T T
+  //    (C[n, q] = sum_m dY[m, n] Thl[m, q]) in one launch; ahead of the dX
+  //    GEMM, which needs only G as well and overlaps this launch
   {
     const int out_bf16 = grad_dtype == QLORA_BF16 ? 1 : 0;
     SkJob ja, jb;
@@ -692,6 +683,22 @@ qlora_status linear_bwd_core(const void* dY, const void* X, const Dims& d, const
     jb.a.transpose = 0;
     jb.a.out = dB;
     st = launch_skinny<1, 1>(ja, &jb, cs);
+    if (st != QLORA_OK) return st;
+  }
+  // 3. dX = dY W^ + (sG) A; under dropout dY W^ in fp32, then one pass
+  //    adding s ((G A) * keep) / (1 - p) and rounding once
+  if (dX && !drop) {
+    st = run_fused(kModeDx, dY, Wq, Wdense, d, sG, A, dX, events, d_status, cs);
+    if (st != QLORA_OK) return st;
+  } else if (dX) {
+    float* dxf = reinterpret_cast<float*>(ws + WD.dxf);
+    st = run_fused(kModeDx, dY, Wq, Wdense, d, sG, A, dX, events, d_status, cs, dxf, false);
+    if (st != QLORA_OK) return st;
+    k_dropout_dx<<<dropout_grid(d.M * (d.K / 8)), kDropThreads, 0, cs>>>(
+        dxf, reinterpret_cast<const float*>(ws + WD.g32), static_cast<const __nv_bfloat16*>(A), d.M, d.K, d.r,
+        s * inv_q, drop->seed, drop->thr, static_cast<__nv_bfloat16*>(dX));
+    st = check_launch();
+    if (st != QLORA_OK) return st;
   }
   return st;
 }

@@ -215,6 +215,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   volatile int* s_last = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // a fused GEMM launched behind this kernel may start its own work now
+  // (it waits for this kernel's results only where it reads them)
+  if (threadIdx.x == 0) griddep_launch_dependents();
   const int64_t p0 = static_cast<int64_t>(ptile) * kSkBM;
   const int q0 = qchunk * 256;
   const int c_begin = split * args.chunks_per_split;
