@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   cluster_sync();   // barriers of both CTAs initialised before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  if (threadIdx.x == 0) QLORA_CHECK_ONLY(Lay::Bytes <= dyn_smem_bytes(), 100);
   auto leader_bar = [&](uint64_t* b) { return mapa_shared(smem_u32(b), 0); };
 
   if (warp == 0) {
@@ -177,7 +178,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * kSlotA);
 #pragma unroll
           for (int t = 0; t < MSUB; ++t)
-            tma_load_2d_pair(smem_u32(slot_a(it)) + t * kPairABytes, &tm_act, fa, it * 64, static_cast<int32_t>(m0 + 256 * t));
+            if (QLORA_CHECK((it % kPairRingA) * kSlotA + (t + 1) * kPairABytes <= Lay::OffW && m0 >= 0, 101))
+              tma_load_2d_pair(smem_u32(slot_a(it)) + t * kPairABytes, &tm_act, fa, it * 64, static_cast<int32_t>(m0 + 256 * t));
         } else {
           // adapter stage: the A tile here; the adapter B tile is loaded into
           // the weight slot, and its bytes counted on that slot's full_w, by
@@ -193,7 +195,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (leader) mbar_arrive_expect_tx(smem_u32(&full_a[ia]), 2 * kSlotA);
 #pragma unroll
           for (int t = 0; t < MSUB; ++t)
-            tma_load_2d_pair(smem_u32(slot_a(it)) + t * kPairABytes, &tm_la, fa, li * 64, static_cast<int32_t>(arow + 256 * t));
+            if (QLORA_CHECK((it % kPairRingA) * kSlotA + (t + 1) * kPairABytes <= Lay::OffW && arow >= 0 && li >= 0, 101))
+              tma_load_2d_pair(smem_u32(slot_a(it)) + t * kPairABytes, &tm_la, fa, li * 64, static_cast<int32_t>(arow + 256 * t));
         }
         ++issued;
       }
@@ -217,6 +220,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const uint32_t fc = smem_u32(&full_c[ic]);
         if (it < args.num_kt && !WDENSE) {
           mbar_arrive_expect_tx(fc, kPairCBytes);
+          if (!QLORA_CHECK(Lay::OffC + (it % kPairRingC + 1) * kPairCBytes <= Lay::OffBar, 102)) {
+            ++issued;   // no load: the wait on this slot runs out (bounded) and the launch aborts
+            continue;
+          }
           if (MODE == kModeFwd)
             tma_load_2d(smem_u32(slot_c(it)), &tm_codes, fc, it * 32, static_cast<int32_t>(nc0));
           else
@@ -245,7 +252,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const int first = (MSUB == 1) ? me : 0;
       constexpr int step = (MSUB == 1) ? kPairIssuers : 1;
       constexpr uint32_t idesc = idesc_bf16(256, 256, 0, MODE == kModeDx ? 1 : 0);
-      for (int it = first; it < total; it += step) {
+      const bool cols_ok = QLORA_CHECK(256u * me + 256u <= kPairTmemCols, 104);
+      for (int it = first; cols_ok && it < total; it += step) {
         const int ia = it % kPairRingA, iw = it % kPairRingW;
         if (!mbar_wait(smem_u32(&full_a[ia]), par(it, kPairRingA), abort_flag, args.status)) break;
         if (!mbar_wait(smem_u32(&full_w[iw]), par(it, kPairRingW), abort_flag, args.status)) break;
@@ -333,7 +341,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const int32_t kk = lora ? ((it - args.num_kt) % nl1) * 64 : it * 64;
           const uint32_t fw = leader_bar(&full_w[iw]);
           mbar_expect_tx_cluster(fw, kPairWBytes);
-          if (MODE == kModeFwd) {
+          // (a skipped load leaves this slot's wait to run out: bounded, the launch aborts)
+          if (!QLORA_CHECK(Lay::OffW + (iw + 1) * kPairWBytes <= Lay::OffC && kk >= 0, 103)) {
+          } else if (MODE == kModeFwd) {
             tma_load_2d_pair(smem_u32(slot_w(it)), map, fw, kk, static_cast<int32_t>(nc0));
           } else {
             tma_load_2d_pair(smem_u32(slot_w(it)), map, fw, static_cast<int32_t>(nc0), kk);
@@ -342,7 +352,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
       } else {
         uint8_t* wdst = slot_w(it) + w_off;
-        if (valid) {
+        if (valid && QLORA_CHECK(Lay::OffW + iw * kPairWBytes + w_off + 128 <= Lay::OffC, 103)) {
           const NF4Table tab = nf4_table(scale);
           const NF4Shr sh = nf4_shr();
           const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -410,6 +420,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int q = warp & 3, j = warp >> 2;
     const uint32_t taddr = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
     uint8_t* stg = base + warp * 8192;
+    const bool stg_ok = QLORA_CHECK(static_cast<uint32_t>(warp + 1) * 8192u <= Lay::OffBar, 106);
     // columns 16 c .. 16 c + 15 (c < 4) of this lane's row of a 64-column box, as bf16
     auto stage16 = [&](uint8_t* box, int c, const uint32_t (&r)[16]) {
       uint32_t pk[8];
@@ -423,7 +434,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     auto store_box = [&](const uint8_t* box, int64_t x, int64_t y) {
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0 && x < args.out_cols && y < args.M) {
+      if (lane == 0 && x < args.out_cols && y < args.M && stg_ok && QLORA_CHECK(x >= 0 && y >= 0 && (x & 7) == 0, 107)) {
         tma_store_2d(&tm_out, smem_u32(box), static_cast<int32_t>(x), static_cast<int32_t>(y));
         bulk_commit();
       }
@@ -436,6 +447,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll 1
       for (int i = 0; i < 4; i += 2) {
         const int col = (4 * j + i) * 16;
+        QLORA_CHECK_ONLY(256 + col + 32 <= static_cast<int>(kPairTmemCols), 105);
         uint32_t r[2][16], r1[2][16];
         tmem_ld16(taddr + col, r[0]);
         tmem_ld16(taddr + 256 + col, r1[0]);
@@ -465,6 +477,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll 1
       for (int bx = 0; bx < 2; ++bx) {
         const int col = (j & 1) * 128 + bx * 64;
+        QLORA_CHECK_ONLY(256 * t + col + 64 <= static_cast<int>(kPairTmemCols), 105);
         uint32_t r[4][16];
 #pragma unroll
         for (int h = 0; h < 4; ++h) tmem_ld16(taddr + 256 * t + col + 16 * h, r[h]);

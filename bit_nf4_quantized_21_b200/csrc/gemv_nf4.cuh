@@ -535,8 +535,10 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         // partial tile: publish, count, and the last arrival adds them up
         const int slot = (u == u0) ? 0 : 1;
         float4* dst = reinterpret_cast<float4*>(args.part + ((c * 2 + slot) * kGvRows + row) * 16);
+        if (QLORA_CHECK(c < kGvMaxCtas && row < kGvRows && t < args.units / KU, 301)) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+        }
         __threadfence();
         named_bar_sync(1, 128);
         const int64_t cf = gv_cta_of(t * KU, U, G), cl = gv_cta_of((t + 1) * KU - 1, U, G);
@@ -553,6 +555,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
           for (int m = 0; m < 16; ++m) y[m] = 0.0f;
           for (int64_t cc = cf; cc <= cl; ++cc) {
             const int sl = (t == gv_begin(cc, U, G) / KU) ? 0 : 1;
+            if (!QLORA_CHECK(cc >= 0 && cc < kGvMaxCtas, 302)) break;
             const float4* src = reinterpret_cast<const float4*>(args.part + ((cc * 2 + sl) * kGvRows + row) * 16);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {

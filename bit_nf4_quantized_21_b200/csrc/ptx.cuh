@@ -28,6 +28,32 @@ namespace qlora {
 // gone on for a while.  Abort-path drains of copies in flight use the same
 // bound, capped at 200 ms.
 __device__ unsigned long long g_qlora_wait_ns = QLORA_WAIT_NS;
+
+// Index-range checks of the debug build (-DQLORA_DEBUG_CHECKS): at the
+// kernels' shared-memory, tensor-memory, workspace and TMA-coordinate
+// computations a check that fails records its site number in
+// g_qlora_range_fail (the first failure is kept) and the access it guards
+// is skipped; nothing traps.  A release build compiles every check to true.
+// The host reads (and clears) the word with qlora_debug_range_check.
+__device__ unsigned int g_qlora_range_fail = 0;
+__device__ __forceinline__ bool qlora_range_ok(bool ok, unsigned int site) {
+  if (!ok) atomicCAS(&g_qlora_range_fail, 0u, site);
+  return ok;
+}
+// bytes of dynamic shared memory this launch was given
+__device__ __forceinline__ uint32_t dyn_smem_bytes() {
+  uint32_t v;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+  return v;
+}
+// QLORA_CHECK guards an access (use its value); QLORA_CHECK_ONLY records.
+#ifdef QLORA_DEBUG_CHECKS
+#define QLORA_CHECK(cond, site) ::qlora::qlora_range_ok((cond), (site))
+#define QLORA_CHECK_ONLY(cond, site) ((void)::qlora::qlora_range_ok((cond), (site)))
+#else
+#define QLORA_CHECK(cond, site) true
+#define QLORA_CHECK_ONLY(cond, site) ((void)0)
+#endif
 __device__ __forceinline__ uint64_t qlora_wait_limit() {
   return *reinterpret_cast<volatile unsigned long long*>(&g_qlora_wait_ns);
 }

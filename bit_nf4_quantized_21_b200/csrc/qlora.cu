@@ -17,6 +17,9 @@
 #include <mutex>
 
 #include "qlora.h"
+#ifndef QLORA_NO_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
 #include "ptx.cuh"
 #include "nf4_constants.cuh"
 #include "nf4_decode.cuh"
@@ -76,6 +79,21 @@ bool bf16_map(CUtensorMap* m, const void* p, uint64_t cols, uint64_t rows, uint6
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p, cols, rows, ld_elems * 2, box_c, box_r,
                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
+
+// A named NVTX range around each enqueueing entry point of the C ABI, so
+// that a timeline tool shows which call enqueued which kernels (header-only
+// NVTX 3: without a tool attached a push or pop checks one pointer).  The
+// no-allocation forward has none.  -DQLORA_NO_NVTX compiles them out.
+struct NvtxRange {
+#ifndef QLORA_NO_NVTX
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+#else
+  explicit NvtxRange(const char*) {}
+#endif
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // kernels with > 48 KB of dynamic shared memory need the opt-in once per device
 bool ensure_smem_attrs() {
@@ -220,6 +238,7 @@ struct SkJob {
 SkinnyArgs sk_args(const SkPlan& pl, float* partial, unsigned int* cnt, int* status) {
   SkinnyArgs a{};
   a.vscale = 1.0f;
+  a.partial_elems = static_cast<int64_t>(pl.partial_bytes / 4);
   a.P = pl.P;
   a.Qn = pl.Qn;
   a.Qtot = pl.Qtot;
@@ -703,6 +722,12 @@ qlora_status linear_bwd_core(const void* dY, const void* X, const Dims& d, const
   return st;
 }
 
+// Records a failed range check at site 0xFFFF without touching memory: the
+// path from a kernel's check to qlora_debug_range_check, in either build.
+__global__ void k_range_selftest() {
+  if (threadIdx.x == 0) qlora::qlora_range_ok(false, 0xFFFFu);
+}
+
 // Validation of the dense-bf16 entries: the same shape rules as the NF4
 // weight (N % 8 == 0, K % 64 == 0, 1 <= r <= 256).
 qlora_status check_dense(int64_t M, const void* W, int64_t N, int64_t K, int r, float alpha, const void* workspace,
@@ -764,6 +789,7 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
 
 qlora_status qlora_quantize_nf4(const void* W, qlora_dtype w_dtype, const qlora_nf4_weight* out, int* d_status,
                                 void* stream) {
+  NvtxRange nvtx_range("qlora_quantize_nf4");
   qlora_status st = check_weight(out, true);
   if (st != QLORA_OK) return st;
   if (!W || !aligned16(W)) return QLORA_ERR_INVALID_ARG;
@@ -784,6 +810,7 @@ qlora_status qlora_quantize_nf4(const void* W, qlora_dtype w_dtype, const qlora_
 }
 
 qlora_status qlora_dequantize(const qlora_nf4_weight* Wq, void* W_out, void* stream) {
+  NvtxRange nvtx_range("qlora_dequantize");
   qlora_status st = check_weight(Wq, true);
   if (st != QLORA_OK) return st;
   if (!W_out || !aligned16(W_out)) return QLORA_ERR_INVALID_ARG;
@@ -798,6 +825,7 @@ qlora_status qlora_dequantize(const qlora_nf4_weight* Wq, void* W_out, void* str
 qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* Wq, const void* A, const void* B,
                               int r, float alpha, void* Y, float* T_save, void* workspace, size_t ws_bytes,
                               int* d_status, const qlora_gemm_events* events, void* stream) {
+  NvtxRange nvtx_range("qlora_linear_fwd");
   qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes);
   if (st != QLORA_OK) return st;
   if (!X || !A || !B || !Y || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y))
@@ -831,6 +859,7 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
                               const void* B, int r, float alpha, const float* T_saved, void* dX, void* dA, void* dB,
                               qlora_dtype grad_dtype, void* workspace, size_t ws_bytes, int* d_status,
                               const qlora_gemm_events* events, void* stream) {
+  NvtxRange nvtx_range("qlora_linear_bwd");
   qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes);
   if (st != QLORA_OK) return st;
   if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
@@ -851,6 +880,7 @@ size_t qlora_workspace_bytes_dropout(int64_t M, int64_t N, int64_t K, int r) {
 }
 
 qlora_status qlora_lora_dropout_mask(int64_t M, int64_t K, double p, uint64_t seed, uint8_t* keep, void* stream) {
+  NvtxRange nvtx_range("qlora_lora_dropout_mask");
   DropCfg c;
   if (!dropout_cfg(p, seed, &c)) return QLORA_ERR_INVALID_ARG;
   if (M < 1 || K < 64 || K % 64 != 0 || M > (int64_t(1) << 31) || K > (int64_t(1) << 31))
@@ -865,6 +895,7 @@ qlora_status qlora_linear_fwd_dropout(const void* X, int64_t M, const qlora_nf4_
                                       const void* B, int r, float alpha, double p, uint64_t seed, void* Y,
                                       float* T_save, void* workspace, size_t ws_bytes, int* d_status,
                                       const qlora_gemm_events* events, void* stream) {
+  NvtxRange nvtx_range("qlora_linear_fwd_dropout");
   qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes, true);
   if (st != QLORA_OK) return st;
   DropCfg drop;
@@ -901,6 +932,7 @@ qlora_status qlora_linear_bwd_dropout(const void* dY, const void* X, int64_t M, 
                                       const float* T_saved, void* dX, void* dA, void* dB, qlora_dtype grad_dtype,
                                       void* workspace, size_t ws_bytes, int* d_status,
                                       const qlora_gemm_events* events, void* stream) {
+  NvtxRange nvtx_range("qlora_linear_bwd_dropout");
   qlora_status st = check_linear(M, Wq, r, alpha, workspace, ws_bytes, true);
   if (st != QLORA_OK) return st;
   DropCfg drop;
@@ -919,6 +951,7 @@ qlora_status qlora_linear_bwd_dropout(const void* dY, const void* X, int64_t M, 
 qlora_status qlora_lora_linear_fwd(const void* X, int64_t M, const void* W, int64_t N, int64_t K, const void* A,
                                    const void* B, int r, float alpha, void* Y, float* T_save, void* workspace,
                                    size_t ws_bytes, int* d_status, const qlora_gemm_events* events, void* stream) {
+  NvtxRange nvtx_range("qlora_lora_linear_fwd");
   qlora_status st = check_dense(M, W, N, K, r, alpha, workspace, ws_bytes);
   if (st != QLORA_OK) return st;
   if (!X || !A || !B || !Y || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y))
@@ -945,6 +978,7 @@ qlora_status qlora_lora_linear_bwd(const void* dY, const void* X, int64_t M, con
                                    const void* A, const void* B, int r, float alpha, const float* T_saved, void* dX,
                                    void* dA, void* dB, qlora_dtype grad_dtype, void* workspace, size_t ws_bytes,
                                    int* d_status, const qlora_gemm_events* events, void* stream) {
+  NvtxRange nvtx_range("qlora_lora_linear_bwd");
   qlora_status st = check_dense(M, W, N, K, r, alpha, workspace, ws_bytes);
   if (st != QLORA_OK) return st;
   if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
@@ -960,6 +994,7 @@ qlora_status qlora_lora_linear_bwd(const void* dY, const void* X, int64_t M, con
 qlora_status qlora_adam_step(float* master, float* m, float* v, void* param_bf16, const void* grad,
                              qlora_dtype grad_dtype, int64_t n, int64_t step, float lr, float beta1, float beta2,
                              float eps, float weight_decay, float grad_scale, int* d_status, void* stream) {
+  NvtxRange nvtx_range("qlora_adam_step");
   if (n < 0 || step < 1) return QLORA_ERR_INVALID_ARG;
   if (grad_dtype != QLORA_F32 && grad_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
   for (float x : {lr, beta1, beta2, eps, weight_decay, grad_scale})
@@ -1006,6 +1041,27 @@ qlora_status qlora_debug_set_pair_mtiles(int n) {
   return QLORA_OK;
 }
 
+int qlora_debug_checks_enabled(void) {
+#ifdef QLORA_DEBUG_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+qlora_status qlora_debug_range_check(unsigned int* site) {
+  if (!site) return QLORA_ERR_INVALID_ARG;
+  *site = 0;
+  const unsigned int zero = 0;
+  if (cudaMemcpyFromSymbol(site, g_qlora_range_fail, sizeof(unsigned int)) != cudaSuccess) return QLORA_ERR_CUDA;
+  return cudaMemcpyToSymbol(g_qlora_range_fail, &zero, sizeof(zero)) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_debug_range_selftest(void* stream) {
+  k_range_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return check_launch();
+}
+
 qlora_status qlora_debug_inject_stall(int on) {
   const int v = on ? 1 : 0;
   return cudaMemcpyToSymbol(g_qlora_inject_stall, &v, sizeof(v)) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
@@ -1040,6 +1096,7 @@ qlora_status qlora_paged_free(void* ptr) {
 }
 
 qlora_status qlora_paged_prefetch(void* ptr, size_t bytes, int to_device, void* stream) {
+  NvtxRange nvtx_range("qlora_paged_prefetch");
   if (!ptr || bytes == 0) return QLORA_ERR_INVALID_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
@@ -1053,6 +1110,7 @@ qlora_status qlora_paged_prefetch(void* ptr, size_t bytes, int to_device, void* 
 
 qlora_status qlora_merge_nf4(const qlora_nf4_weight* Wq, const void* A, const void* B, int r, float alpha,
                              float* W_merged, const qlora_nf4_weight* out, int* d_status, void* stream) {
+  NvtxRange nvtx_range("qlora_merge_nf4");
   qlora_status st = check_weight(Wq, true);
   if (st != QLORA_OK) return st;
   st = check_weight(out, true);

@@ -51,6 +51,7 @@ struct SkinnyArgs {
   int stages;
   int ptiles, splits, qchunks;   // CTA grid of this problem: ptiles x splits x qchunks
   float* partial;     // [splits][P][Qtot], used when splits * qchunks > 1
+  int64_t partial_elems;   // floats the partial buffer holds (range checks of the debug build)
   unsigned int* cnt;  // [ptiles] arrival counters, zero on entry (when splits * qchunks > 1)
   int* status;
   // the final transform
@@ -245,6 +246,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  if (threadIdx.x == 0)
+    QLORA_CHECK_ONLY(static_cast<uint32_t>(S) * stage_bytes + (2 * S + 1) * 8 + 16 + 1023 <= dyn_smem_bytes(), 200);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -331,6 +334,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         if (rows_mode) {
 #pragma unroll 1
           for (int c = 0; c < args.r16 / 16; ++c) {
+            if (!QLORA_CHECK(static_cast<uint32_t>(c * 16 + 16) <= tcols, 202)) break;
             uint32_t t[16];
             tmem_ld16(taddr + c * 16, t);
             tmem_ld_wait();
@@ -342,6 +346,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         } else {
 #pragma unroll 1
           for (int c = 0; c < args.r16 / 16; ++c) {
+            if (!QLORA_CHECK(static_cast<uint32_t>(args.r16 + c * 16 + 16) <= tcols, 202)) break;
             uint32_t th[16], tl[16];
             tmem_ld16(taddr + c * 16, th);
             tmem_ld16(taddr + args.r16 + c * 16, tl);
@@ -361,7 +366,10 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           uint32_t t[16];
           tmem_ld16(taddr + c * 16, t);
           tmem_ld_wait();
-          if (row < args.P) {
+          if (row < args.P &&
+              QLORA_CHECK(static_cast<uint32_t>(c * 16 + 16) <= tcols &&
+                              (static_cast<int64_t>(split) * args.P + row) * args.Qtot + q0 + c * 16 + 16 <= args.partial_elems,
+                          201)) {
             float4* d4 = reinterpret_cast<float4*>(dst + c * 16);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -381,7 +389,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           __threadfence();
           const float* src = args.partial + row * args.Qtot;
           const int64_t sstride = args.P * args.Qtot;
-          if (row < args.P) {
+          [[maybe_unused]] const int need = rows_mode ? args.r16 : 2 * args.r16;
+          if (row < args.P &&
+              QLORA_CHECK((args.splits - 1) * sstride + row * args.Qtot + need <= args.partial_elems, 203)) {
 #pragma unroll 1
             for (int c = 0; c < args.r16 / 16; ++c) {
               // The partials come from L2: loads of several splits are put in

@@ -16,7 +16,9 @@ from dataclasses import dataclass
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libqlora.so")
+# the library to load: libqlora.so, or another build of it (the debug build
+# with index-range checks, libqlora_debug.so) named by QLORA_LIB
+LIB_PATH = os.environ.get("QLORA_LIB") or os.path.join(_PKG, "libqlora.so")
 
 QLORA_OK = 0
 QLORA_F32 = 0
@@ -31,7 +33,8 @@ EXPORTED = (
     "qlora_adam_step", "qlora_merge_nf4", "qlora_workspace_bytes_dropout", "qlora_lora_dropout_mask",
     "qlora_linear_fwd_dropout", "qlora_linear_bwd_dropout", "qlora_paged_alloc", "qlora_paged_free",
     "qlora_paged_prefetch", "qlora_debug_set_wait_limit", "qlora_debug_inject_stall",
-    "qlora_debug_set_pair_mtiles",
+    "qlora_debug_set_pair_mtiles", "qlora_debug_checks_enabled", "qlora_debug_range_check",
+    "qlora_debug_range_selftest",
 )
 
 
@@ -133,6 +136,12 @@ def lib() -> ctypes.CDLL:
             L.qlora_debug_inject_stall.restype = I32
             L.qlora_debug_set_pair_mtiles.argtypes = [I32]
             L.qlora_debug_set_pair_mtiles.restype = I32
+            L.qlora_debug_checks_enabled.argtypes = []
+            L.qlora_debug_checks_enabled.restype = I32
+            L.qlora_debug_range_check.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+            L.qlora_debug_range_check.restype = I32
+            L.qlora_debug_range_selftest.argtypes = [P]
+            L.qlora_debug_range_selftest.restype = I32
             L.qlora_status_string.argtypes = [I32]
             L.qlora_status_string.restype = ctypes.c_char_p
             L.qlora_version.argtypes = []

@@ -357,6 +357,25 @@ qlora_status qlora_debug_inject_stall(int on);
 qlora_status qlora_debug_set_pair_mtiles(int n);
 
 /*
+ * Index-range checks (no counterpart on the pages).  A library built with
+ * -DQLORA_DEBUG_CHECKS (libqlora_debug.so) checks its kernels' shared-
+ * memory, tensor-memory, workspace and TMA-coordinate computations; a
+ * failed check records the number of its site in a device word (the first
+ * failure is kept) and skips the access it guards, never traps; a launch
+ * whose load was skipped then ends by a timed-out wait
+ * (QLORA_DEV_TIMEOUT_BIT).  The release library compiles the checks out.
+ *   qlora_debug_checks_enabled: 1 in the debug build, else 0.
+ *   qlora_debug_range_check(site): *site = that word (0: no failure since
+ *     the last read), then clears it; synchronous.
+ *   qlora_debug_range_selftest(stream): enqueues a kernel that records a
+ *     failure at site 0xFFFF without touching memory (either build), so a
+ *     test can check the path from a kernel to the host.
+ */
+int qlora_debug_checks_enabled(void);
+qlora_status qlora_debug_range_check(unsigned int* site);
+qlora_status qlora_debug_range_selftest(void* stream);
+
+/*
  * Paged optimiser state ("QLoRA", learning-llms page, the paragraph on paged
  * optimizers; "QLoRA", scalata.ai, "How it works": optimiser state kept in
  * unified memory, which the driver pages out to host RAM when a memory
