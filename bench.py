@@ -849,6 +849,22 @@ def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_param
     out["merge"] = {"value": round(mbytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "shape": [p["N"], p["K"]],
                     "us": round(ms * 1e3, 2), "frac_of_hbm": round(mbytes / (ms * 1e-3) / 1e9 / hbm, 4)}
     assert layer.status.item() == 0, f"device status {layer.status.item()}"
+    # the same merge in one pass, merged weights formed in registers (no fp32
+    # buffer): bytes per weight NF4 read 0.516 + NF4 write 0.516, plus A and
+    # B once; its 2 r fp32 operations per weight for the product B A bound it
+    # by arithmetic before bandwidth
+    f1 = lambda: q.qlora_merge_nf4(p["Wq"], p["A"], p["B"], layer.wl.alpha, out=Wnew, keep_merged=False,
+                                   d_status=layer.status)
+    for _ in range(3):
+        f1()
+    ms1 = statistics.median(time_events(f1, 10, flush=lambda: l2buf.add_(1)))
+    fbytes = 2 * p["Wq"].nbytes() + 2 * (p["A"].numel() + p["B"].numel())
+    out["merge_fused"] = {"value": round(fbytes / (ms1 * 1e-3) / 1e9, 1), "unit": "GB/s",
+                          "shape": [p["N"], p["K"]], "us": round(ms1 * 1e3, 2),
+                          "frac_of_hbm": round(fbytes / (ms1 * 1e-3) / 1e9 / hbm, 4),
+                          "fp32_ops_per_s": round(4 * p["A"].shape[0] * p["N"] * p["K"] / (ms1 * 1e-3), 1),
+                          "time_vs_two_pass": round(ms1 / ms, 4)}
+    assert layer.status.item() == 0, f"device status {layer.status.item()}"
     del Wm, Wnew
     # plain LoRA on a bf16 base (the weights' dequantised copies) through the
     # same GEMM, timed with the same harness as the NF4 step beside it: the

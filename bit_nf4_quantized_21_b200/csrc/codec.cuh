@@ -88,6 +88,16 @@ __device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
   return static_cast<uint32_t>(r) & 0xFFu;
 }
 
+// Where the weights come from: a bf16 or fp32 matrix in global memory
+// (the quantiser), or values a source computes itself (the fused adapter
+// merge, merge.cuh).  load(e0) returns the 16 weights e0 .. e0 + 15 of one
+// block in a form widen16 / mag_bits16 accept.
+template <typename T> struct PtrSrc {
+  const T* p;
+  static constexpr int kMinBlocks = sizeof(T) == 2 ? 4 : 3;   // CTAs per SM the registers allow
+  __device__ __forceinline__ Raw16<T> load(int64_t e0) const { return load_raw16(p + e0); }
+};
+
 // K1.  Grid: one CTA per group of 256 blocks (16384 weights).  Four threads
 // share a 64-weight block (16 weights each, two 16-byte loads of bf16), so a
 // warp reads 8 whole blocks = 1 KB contiguous and writes 256 contiguous
@@ -97,9 +107,9 @@ __device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
 // any is used and are kept as loaded (32 registers for bf16); 4 CTAs per SM
 // keep 128 B per thread, 128 KB per SM, in flight.
 // The encoding is ~10 instructions per weight.
-template <typename T>
-__global__ void __launch_bounds__(kQuantThreads, sizeof(T) == 2 ? 4 : 3)
-    k_quantize_nf4(const T* __restrict__ w, int64_t nblocks, int dq, uint8_t* __restrict__ codes,
+template <typename Src>
+__global__ void __launch_bounds__(kQuantThreads, Src::kMinBlocks)
+    k_quantize_nf4(const Src src, int64_t nblocks, int dq, uint8_t* __restrict__ codes,
                    uint8_t* __restrict__ q8, float* __restrict__ s2,
                    float* __restrict__ absmax_out, int* status) {
   __shared__ NF4CellTable s_cell;
@@ -117,11 +127,11 @@ __global__ void __launch_bounds__(kQuantThreads, sizeof(T) == 2 ? 4 : 3)
   const int sub = tid & 3;   // weights 16 sub .. 16 sub + 15 of the block
   bool nonfinite = false;
 
-  Raw16<T> raw[4];
+  decltype(src.load(0)) raw[4];
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
     const int lb = it * 64 + (tid >> 2);
-    if (lb < nb) raw[it] = load_raw16(w + (b0 + lb) * 64 + sub * 16);
+    if (lb < nb) raw[it] = src.load((b0 + lb) * 64 + sub * 16);
   }
   __syncthreads();   // the cell table is in shared memory
 #pragma unroll

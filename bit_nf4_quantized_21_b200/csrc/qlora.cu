@@ -799,13 +799,13 @@ qlora_status qlora_quantize_nf4(const void* W, qlora_dtype w_dtype, const qlora_
   const unsigned groups = static_cast<unsigned>(cdiv(nblocks, 256));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (w_dtype == QLORA_BF16)
-    k_quantize_nf4<__nv_bfloat16><<<groups, kQuantThreads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(W), nblocks, out->double_quant, out->codes, out->absmax_q8,
-        out->group_scale, out->absmax_f32, d_status);
+    k_quantize_nf4<<<groups, kQuantThreads, 0, s>>>(
+        PtrSrc<__nv_bfloat16>{static_cast<const __nv_bfloat16*>(W)}, nblocks, out->double_quant, out->codes,
+        out->absmax_q8, out->group_scale, out->absmax_f32, d_status);
   else
-    k_quantize_nf4<float><<<groups, kQuantThreads, 0, s>>>(static_cast<const float*>(W), nblocks,
-                                                           out->double_quant, out->codes, out->absmax_q8,
-                                                           out->group_scale, out->absmax_f32, d_status);
+    k_quantize_nf4<<<groups, kQuantThreads, 0, s>>>(PtrSrc<float>{static_cast<const float*>(W)}, nblocks,
+                                                    out->double_quant, out->codes, out->absmax_q8,
+                                                    out->group_scale, out->absmax_f32, d_status);
   return check_launch();
 }
 
@@ -1118,10 +1118,20 @@ qlora_status qlora_merge_nf4(const qlora_nf4_weight* Wq, const void* A, const vo
   if (out->rows != Wq->rows || out->cols != Wq->cols) return QLORA_ERR_INVALID_ARG;
   if (out->absmax_f32 && !aligned16(out->absmax_f32)) return QLORA_ERR_INVALID_ARG;
   if (r < 1 || r > 256 || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
-  if (!A || !B || !W_merged || !aligned16(A) || !aligned16(B) || !aligned16(W_merged)) return QLORA_ERR_INVALID_ARG;
+  if (!A || !B || !aligned16(A) || !aligned16(B) || (W_merged && !aligned16(W_merged))) return QLORA_ERR_INVALID_ARG;
   const int64_t N = Wq->rows, K = Wq->cols;
   const float s = alpha / static_cast<float>(r);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (!W_merged) {
+    // one pass: the quantiser kernel forms each merged weight itself
+    if (out->codes == Wq->codes) return QLORA_ERR_INVALID_ARG;   // in place needs the two-pass form
+    const int64_t nblocks = N * K / 64;
+    const qlora::MergeSrc src{Wq->codes, Wq->absmax_q8, Wq->group_scale, Wq->absmax_f32, Wq->double_quant, K,
+                              static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), r, s};
+    qlora::k_quantize_nf4<<<static_cast<unsigned>(cdiv(nblocks, 256)), qlora::kQuantThreads, 0, cs>>>(
+        src, nblocks, out->double_quant, out->codes, out->absmax_q8, out->group_scale, out->absmax_f32, d_status);
+    return check_launch();
+  }
   const int64_t threads = N * (K / 8);
   qlora::k_merge_nf4<<<static_cast<unsigned>(cdiv(threads, qlora::kMergeThreads)), qlora::kMergeThreads, 0, cs>>>(
       Wq->codes, Wq->absmax_q8, Wq->group_scale, Wq->absmax_f32, Wq->double_quant, N, K,

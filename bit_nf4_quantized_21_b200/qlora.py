@@ -250,14 +250,19 @@ def qlora_quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, double_qua
 
 def qlora_merge_nf4(Wq: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
                     out: NF4Weight | None = None, W_merged: torch.Tensor | None = None,
-                    double_quant: bool = True, d_status: torch.Tensor | None = None, stream=None):
+                    double_quant: bool = True, d_status: torch.Tensor | None = None, stream=None,
+                    keep_merged: bool = True):
     """NF4(W^ + (alpha/r) B A) into `out` (new, or Wq itself for in place);
-    returns (out, W_merged) with W_merged the fp32 merged weight."""
+    returns (out, W_merged) with W_merged the fp32 merged weight.  With
+    keep_merged=False the merge is one fused pass (no fp32 buffer; not in
+    place) and W_merged is None."""
     r = A.shape[0]
     dev = Wq.codes.device
     if out is None:
         out = empty_nf4(Wq.rows, Wq.cols, dev, double_quant)
-    if W_merged is None:
+    if not keep_merged:
+        W_merged = None
+    elif W_merged is None:
         W_merged = torch.empty((Wq.rows, Wq.cols), dtype=torch.float32, device=dev)
     cw, co = Wq.c(), out.c()
     _check(lib().qlora_merge_nf4(ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha), _ptr(W_merged),

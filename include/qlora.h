@@ -288,13 +288,18 @@ qlora_status qlora_lora_linear_bwd(const void* dY, const void* X, int64_t M, con
  * re-quantisation; katajob.com, "What it costs": merge friction).  Each
  * merged weight is formed in fp32, every operation rounded once, in this
  * order:  acc = 0; for j = 0..r-1: acc = acc + B[n,j] * A[j,k];
- * W'[n,k] = W^[n,k] + s * acc  (W^ the bf16 dequantised weight), written
- * to W_merged (fp32 [N, K], caller-provided scratch, left holding W'),
- * then quantised into `out` exactly as qlora_quantize_nf4 would quantise
- * W_merged.  A bf16 [r, K], B bf16 [N, r]; 1 <= r <= 256.  `out` has
- * Wq's rows and cols, its own double_quant setting, and may be Wq itself
- * (the two launches are ordered on the stream).  Non-finite merged values
- * set QLORA_DEV_NONFINITE_BIT as in the quantiser.
+ * W'[n,k] = W^[n,k] + s * acc  (W^ the bf16 dequantised weight), and
+ * quantised into `out` exactly as qlora_quantize_nf4 would quantise W'
+ * held in fp32.  A bf16 [r, K], B bf16 [N, r]; 1 <= r <= 256.  `out` has
+ * Wq's rows and cols and its own double_quant setting.  Two forms:
+ *   W_merged non-NULL (fp32 [N, K], 16-byte aligned, caller-provided):
+ *     W' is written there and left holding it, then quantised by a second
+ *     launch; `out` may be Wq itself (the launches are ordered on the
+ *     stream).
+ *   W_merged NULL: one launch forms W' in registers and quantises it (the
+ *     same codes and scales bit for bit, without the fp32 round trip);
+ *     `out` must not share Wq's codes (QLORA_ERR_INVALID_ARG).
+ * Non-finite merged values set QLORA_DEV_NONFINITE_BIT as in the quantiser.
  */
 qlora_status qlora_merge_nf4(const qlora_nf4_weight* Wq, const void* A, const void* B, int r,
                              float alpha, float* W_merged, const qlora_nf4_weight* out,

@@ -229,7 +229,7 @@ def linear_bwd(dY, X, W_hat, A, B, alpha: float, r: int, T=None):
     return {"dX": dX, "dA": dA, "dB": dB, "G": G, "T": T}
 
 
-def merge_nf4(q: dict, A, B, alpha: float, r: int) -> np.ndarray:
+def merge_nf4(q: dict, A, B, alpha: float, r: int, W_hat=None) -> np.ndarray:
     """The merged weight W^ + s B A as fp32 [N, K], before re-quantisation
     ("QLoRA", learning-llms page, the fine-print bullet on merging: adding
     the bf16 update into 4-bit weights forces a re-quantisation).  The pages
@@ -237,8 +237,10 @@ def merge_nf4(q: dict, A, B, alpha: float, r: int) -> np.ndarray:
     takes the library's precision and order: fp32, every operation rounded
     once, acc = sum over j of B[:, j] * A[j, :] in j order, then W^ + s acc
     with s = fp32(alpha) / fp32(r).  numpy float32 arithmetic rounds each
-    operation (no fused multiply-add)."""
-    W = bf16_to_f32(nf4_dequantize(q)).astype(np.float32)
+    operation (no fused multiply-add).  W_hat: the dequantised weight as
+    bf16 bits, for a source in another scale format (default: decoded from
+    q with nf4_dequantize)."""
+    W = bf16_to_f32(nf4_dequantize(q) if W_hat is None else np.asarray(W_hat, np.uint16)).astype(np.float32)
     a = bf16_to_f32(np.asarray(A, np.uint16)).astype(np.float32)
     b = bf16_to_f32(np.asarray(B, np.uint16)).astype(np.float32)
     s = np.float32(alpha) / np.float32(r)
