@@ -48,7 +48,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one fused-GEMM launch (gate forward) from the ncu capture
 # summarised in profiles/k_gemm_nf4_pair_fwd_gate_m2048.md; None once the
 # kernel changes and until it is captured again.
-GEMM_TRAFFIC_BYTES = 48.94e6
+GEMM_TRAFFIC_BYTES = 51.67e6
 
 
 def step_flops(wl=WL, M=None) -> float:

@@ -188,17 +188,17 @@ __device__ __forceinline__ float gv_dot8(uint4 x, uint4 a, float acc) {
   return acc;
 }
 
-// The 128 epilogue threads of this CTA publish their writes (fence, then one
-// arrival on the grid counter) and wait until all G CTAs have arrived.
-// Bounded: on timeout the CTA's abort flag and the timeout status are set.
-// Returns the same outcome in every one of the 128 threads.
+// The 128 epilogue threads of this CTA publish their writes (a barrier, then
+// one releasing arrival on the grid counter) and wait until all G CTAs have
+// arrived (an acquiring poll, then a barrier).  Bounded: on timeout the
+// CTA's abort flag and the timeout status are set.  Returns the same
+// outcome in every one of the 128 threads.
 __device__ __forceinline__ bool gv_grid_arrive_wait(int* ctr, int64_t G, int et, volatile int* abort_flag,
                                                     int* status) {
-  __threadfence();
   named_bar_sync(1, 128);
   bool ok = true;
   if (et == 0) {
-    atomicAdd(ctr, 1);
+    red_add_release_gpu(ctr, 1);
     const uint64_t t0 = global_ns();
     while (true) {
       int v;
@@ -215,7 +215,6 @@ __device__ __forceinline__ bool gv_grid_arrive_wait(int* ctr, int64_t G, int et,
     }
   }
   ok = named_bar_and(1, 128, ok);
-  __threadfence();
   return ok;
 }
 
@@ -539,18 +538,15 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
         }
-        __threadfence();
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 128);   // every partial write of the CTA before the release below
         const int64_t cf = gv_cta_of(t * KU, U, G), cl = gv_cta_of((t + 1) * KU - 1, U, G);
         if (et == 0) {
-          __threadfence();
-          const int old = atomicAdd(args.cnt + t, 1);
+          const int old = static_cast<int>(atom_add_acq_rel_gpu(reinterpret_cast<unsigned int*>(args.cnt + t), 1u));
           *s_last = (old == static_cast<int>(cl - cf)) ? 1 : 0;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 128);   // the acquire above before any partial read of the CTA
         finish = *s_last != 0;
         if (finish) {
-          __threadfence();
 #pragma unroll
           for (int m = 0; m < 16; ++m) y[m] = 0.0f;
           for (int64_t cc = cf; cc <= cl; ++cc) {

@@ -40,6 +40,21 @@ __device__ __forceinline__ bool qlora_range_ok(bool ok, unsigned int site) {
   if (!ok) atomicCAS(&g_qlora_range_fail, 0u, site);
   return ok;
 }
+// Atomic add at GPU scope with acquire-release semantics.  After a CTA
+// barrier, one thread's release publishes the writes every thread of the
+// CTA made before the barrier (release is cumulative); the thread whose add
+// sees the final count acquires every write released by the others, and a
+// CTA barrier after it extends that to its whole CTA.  This replaces a
+// fence per thread around a split-K arrival.
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // bytes of dynamic shared memory this launch was given
 __device__ __forceinline__ uint32_t dyn_smem_bytes() {
   uint32_t v;

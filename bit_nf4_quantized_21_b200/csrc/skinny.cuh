@@ -359,10 +359,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           }
         }
       } else {
-        // publish this CTA's partial tile, count in, the last arrival finishes
+        // publish this CTA's partial tile, count in, the last arrival finishes;
+        // only the columns the finish reads (r16 of T or G; the hi and lo
+        // halves, 2 r16, of dA or dB) -- Qn is rounded up to a whole box
         float* dst = args.partial + (static_cast<int64_t>(split) * args.P + row) * args.Qtot + q0;
+        const int used = min(qv, max(0, (rows_mode ? args.r16 : 2 * args.r16) - q0));
 #pragma unroll 1
-        for (int c = 0; c < qv / 16; ++c) {
+        for (int c = 0; c < used / 16; ++c) {
           uint32_t t[16];
           tmem_ld16(taddr + c * 16, t);
           tmem_ld_wait();
@@ -377,16 +380,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
                                   __uint_as_float(t[4 * i + 2]), __uint_as_float(t[4 * i + 3]));
           }
         }
-        __threadfence();
-        sk_bar(128);
+        sk_bar(128);   // every partial write of the CTA before the release below
         if (et == 0) {
-          __threadfence();
-          const unsigned int old = atomicAdd(args.cnt + ptile, 1u);
+          const unsigned int old = atom_add_acq_rel_gpu(args.cnt + ptile, 1u);
           *s_last = (old == static_cast<unsigned int>(nred - 1)) ? 1 : 0;
         }
-        sk_bar(128);
+        sk_bar(128);   // the acquire above before any partial read of the CTA
         if (*s_last) {
-          __threadfence();
           const float* src = args.partial + row * args.Qtot;
           const int64_t sstride = args.P * args.Qtot;
           [[maybe_unused]] const int need = rows_mode ? args.r16 : 2 * args.r16;
