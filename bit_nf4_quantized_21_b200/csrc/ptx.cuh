@@ -113,21 +113,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test: unlike try_wait, which may suspend the thread for a
-// while when the phase is incomplete, test_wait returns at once -- for a
-// thread that polls several barriers and must not stall on any one.
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait.  `abort_flag` is a CTA-shared word: once any role has given
 // up, the others stop waiting too.  Returns false on timeout/abort.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
@@ -144,36 +129,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
         if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
         return false;
       }
-    }
-  }
-}
-
-// try_wait with a suspend-time hint: a thread whose phase is incomplete is
-// suspended (issuing nothing) for up to `ns` or until the phase completes.
-__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.b32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(ns)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait built on the hinted try_wait (for a thread whose polling
-// would take issue slots from busy warps on its scheduler).
-__device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                               int* status, uint32_t ns) {
-  if (mbar_try_wait_hint(bar, parity, ns)) return true;
-  const uint64_t t0 = global_ns();
-  while (true) {
-    if (mbar_try_wait_hint(bar, parity, ns)) return true;
-    if (*abort_flag) return false;
-    if (global_ns() - t0 > qlora_wait_limit()) {
-      *abort_flag = 1;
-      if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
-      return false;
     }
   }
 }
@@ -374,25 +329,6 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
       : "memory");
   return ok != 0;
 }
-// Bounded wait with cluster-scope acquire (for barriers other CTAs arrive on).
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                                  int* status) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  uint32_t spins = 0;
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((++spins & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > qlora_wait_limit()) {
-        *abort_flag = 1;
-        if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
 // 2-D tiled TMA load issued by either CTA of a 2-SM pair; the transaction
 // bytes complete on the barrier at cluster address `bar_cluster` (the
 // leader's).  No multicast.
