@@ -497,8 +497,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
     }
   }
-  // the TMA stores have read their shared-memory boxes (and landed) before the CTA can exit
-  if (args.tma_out && lane == 0) bulk_wait_all();
+  // the TMA stores have read their shared-memory boxes before the CTA can exit
+  if (args.tma_out && lane == 0) bulk_wait_read();
 
   // this grid does not complete before the kernel ahead of it (when no
   // adapter stage waited for it above)

@@ -171,7 +171,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 }
 
 // 2-D tiled store of a shared-memory box to global memory (bulk async
-// group; commit with bulk_commit, wait with bulk_wait_all).  Elements of the
+// group; commit with bulk_commit, wait with bulk_wait_read).  Elements of the
 // box outside the tensor are not written.  c0 * elemsize must be a multiple
 // of 16 bytes; callers pass non-negative coordinates inside the tensor.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t c0, int32_t c1) {
@@ -181,8 +181,10 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// every bulk store this thread committed has completed
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// every bulk store this thread committed has read its shared-memory source
+// (the shared memory may be reused or released; the global writes complete
+// before the grid does)
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // Programmatic dependent launch.  A kernel launched with programmatic
 // stream serialisation may start before the kernel ahead of it in the
