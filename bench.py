@@ -954,7 +954,51 @@ def sub_measurements(q, dev, peaks, l2buf, layer, quant_ms, quant_bytes, n_param
                         "kernel_frac_of_hbm": round(sum(kgbs) / len(kgbs) / hbm, 4)}
     out["decode_gemv"] = {"unit": "GB/s of NF4 weight (121.17 MB per matrix)", **dec,
                           "peak_hbm_gbs": hbm}
-    del mats
+    # a token's pass through one 70B layer's MLP: gate, up and down decoded
+    # back to back with no flush -- each matrix was last read two 121 MB
+    # matrices earlier, more than L2 holds (L2 defeated by rotating the
+    # weights instead of a flush), and each call's launch overlaps the one
+    # before it as in a model's decode
+    name, N, K = wl.shapes[0]
+    seed = inputs.matrix_seed(wl.base_seed, 0, 2)
+    Wu = inputs.weight((N, K), wl.w_std, seed, device=dev, outlier_frac=wl.outlier_frac,
+                       outlier_scale=wl.outlier_scale)
+    up = ("up", N, K, q.qlora_quantize_nf4(Wu), inputs.normal((wl.r, K), 0.01, seed * 16 + 3, dev),
+          inputs.normal((N, wl.r), 0.01, seed * 16 + 4, dev))
+    del Wu
+    seq = [mats[0], up, mats[1]]
+    seq_bytes = sum(m[3].nbytes() for m in seq)
+    mlp = {}
+    for M in inputs.DECODE_M:
+        calls = []
+        for name, N, K, Wq, A, B in seq:
+            X = inputs.normal((M, K), 1.0, 99 + M, dev)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(q.qlora_workspace_bytes(M, N, K, wl.r), dtype=torch.uint8, device=dev)
+            calls.append((X, Wq, A, B, Y, ws))
+
+        def token_pass():
+            for X, Wq, A, B, Y, ws in calls:
+                q.qlora_linear_fwd(X, Wq, A, B, wl.alpha, Y=Y, workspace=ws)
+        for _ in range(3):
+            token_pass()
+        reps = 10
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(1_000_000)   # the passes are queued before the start event is reached
+        e0.record()
+        for _ in range(reps):
+            token_pass()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        gbs = seq_bytes / (us * 1e-6) / 1e9
+        mlp[f"M{M}"] = {"us_per_pass": round(us, 2), "weight_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / hbm, 4)}
+        del calls
+    out["decode_mlp_pass"] = {"unit": "GB/s of NF4 weight over gate, up and down (363.5 MB)",
+                              "weights": "70B MLP matrices 28672 x 8192 (gate, up) and 8192 x 28672 (down)",
+                              "l2": "defeated by rotating the three matrices (no flush)", **mlp}
+    del mats, seq, up
     torch.cuda.empty_cache()
     out.update(config_workloads(q, dev, hbm))
     return out
